@@ -1,0 +1,77 @@
+"""Softmax attention in fp64 (oracle; test infrastructure only).
+
+Self-attention: Wan2.2 source reading, ch. 4, section "Full forward of one
+block" -- full 3D joint attention, every token of every frame attends to
+every other token with no mask (the intro of ch. 4 chooses full joint
+attention over factorised attention); ch. 8 "What is 75600^2" counts its two
+matrix products QK^T and AV.
+
+Cross-attention: Wan2.2 source reading, ch. 3 "Where did the prompt go" --
+video tokens are the queries, the text context gives keys/values, and each
+prompt is trimmed to its true length ``u[:v]`` with
+``seq_lens = mask.gt(0).sum(dim=1)``; the forward passes ``context_lens`` on
+to ``cross_attn``.  Wan paper explainer, section "Text encoder": the
+cross-attention is ``softmax(Q K_text^T / sqrt(d_k)) V_text``.
+
+Definition evaluated here, for each batch row b and head h:
+
+    s_ij = (q_i . k_j) * scale,   j < kv_len
+    m_i  = max_j s_ij
+    p_ij = exp(s_ij - m_i)
+    o_i  = sum_j p_ij v_j / sum_j p_ij
+
+in float64 with no intermediate rounding beyond fp64's own.  Keys at or
+beyond kv_len take no part (their contents never enter the arithmetic).
+Rows are independent, so evaluating a subset of query rows (``rows=``) or
+evaluating rows in groups to bound memory changes no row's definition; the
+library matmul may only sum in another order (fp64 rounding level).
+"""
+
+import numpy as np
+
+
+def softmax_rows(s):
+    """Row softmax of a float64 score matrix (max-subtracted exp / sum)."""
+    m = s.max(axis=1, keepdims=True)
+    p = np.exp(s - m)
+    return p / p.sum(axis=1, keepdims=True)
+
+
+def attend(q, k, v, scale, kv_len=None):
+    """One (batch, head) slice: q [Lq, d], k/v [Lk, d] -> o [Lq, d] fp64."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    if kv_len is not None:
+        if not 1 <= kv_len <= k.shape[0]:
+            raise ValueError("kv_len out of range")
+        k = k[:kv_len]
+        v = v[:kv_len]
+    s = (q @ k.T) * scale
+    return softmax_rows(s) @ v
+
+
+def attention(q, k, v, scale, kv_lens=None, rows=None, row_block=512):
+    """Batched attention over [B, L, heads, d] tensors.
+
+    q: [B, Lq, heads, d]; k, v: [B, Lk, heads, d]; kv_lens: per-batch valid
+    key count (None = all Lk keys); rows: optional 1-D array of query indices
+    to evaluate (default all).  Returns [B, len(rows), heads, d] float64.
+    """
+    q = np.asarray(q)
+    k = np.asarray(k)
+    v = np.asarray(v)
+    b_, lq, nh, d = q.shape
+    rows = np.arange(lq) if rows is None else np.asarray(rows)
+    out = np.empty((b_, rows.shape[0], nh, d), dtype=np.float64)
+    for b in range(b_):
+        kv_len = None if kv_lens is None else int(kv_lens[b])
+        for h in range(nh):
+            kh = k[b, :, h, :].astype(np.float64)
+            vh = v[b, :, h, :].astype(np.float64)
+            for r0 in range(0, rows.shape[0], row_block):
+                sel = rows[r0:r0 + row_block]
+                qh = q[b, sel, h, :].astype(np.float64)
+                out[b, r0:r0 + row_block, h, :] = attend(qh, kh, vh, scale,
+                                                         kv_len)
+    return out
