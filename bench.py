@@ -1,0 +1,417 @@
+#!/usr/bin/env python
+"""Benchmark of the Wan DiT hot path on B200.
+
+One step = one pass of the whole hot path over one batch of synthetic input
+of the named workload: 3D RoPE (fused into the self-attention tile stage, or
+as its own pass with --rope pre), full spatio-temporal self-attention,
+length-masked cross-attention to 512 text tokens (queried by the
+self-attention output), and the fused CFG + Euler step on the latent, with
+the token grid and sigma schedule from the library's host calls.
+
+Metric: self-attention TFLOP/s (4 * B * heads * L^2 * 128 FLOP per step)
+over the whole step time; also reported against the measured dense bf16
+peak.  Inputs (Q, K, V: 774 MB each at 75,600 tokens x 40 heads) are larger
+than L2, so no flush is needed between steps.
+
+Usage:  python bench.py [--gpus N] [--steps K] [--warmup W]
+        [--workload 720p-81f|480p-81f|...] [--rope fused|pre]
+        [--impl wan|reference]
+Multi-GPU (weak scaling, independent problem per rank, no data-path
+collective): python -m torch.distributed.run --nproc-per-node N bench.py
+--gpus N ...
+"""
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+HOST_GBS_FALLBACK = None
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--workload", default="720p-81f")
+    p.add_argument("--rope", choices=["fused", "pre"], default="pre")
+    p.add_argument("--impl", choices=["wan", "reference"], default="wan")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-rows", type=int, default=4096,
+                   help="query rows of one head timed on the oracle")
+    return p.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0,
+                "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info()
+             if i.get("user_api") == "blas"]
+        if n:
+            return max(n)
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,"
+              "clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(device_index),
+                 "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                 "sw_power_cap"]
+        for line in out.splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[3:7]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------- reference ---
+
+def cpu_oracle_sample(w, rows, seed_rank=0):
+    """Time the oracle (fp64 CPU) on `rows` query rows of one head of the
+    workload: 3D RoPE of that head's Q rows and all K, then softmax
+    attention against all L keys.  Returns (seconds, flops, sample text)."""
+    import numpy as np
+    from oracle import attention as oattn
+    from oracle import grid as ogrid
+    from oracle import rope as orope
+    from video_diffusion_transformer_self_b200 import inputs
+
+    grid = ogrid.token_grid(w.frames, w.height, w.width)
+    L = ogrid.token_count(grid)
+    shape = (1, L, 1, 128)
+    q = inputs.randn_bf16(shape, inputs.seed_for(w.index, "q")).double().numpy()
+    k = inputs.randn_bf16(shape, inputs.seed_for(w.index, "k")).double().numpy()
+    v = inputs.randn_bf16(shape, inputs.seed_for(w.index, "v")).double().numpy()
+    sel = inputs.sample_rows(L, rows, inputs.seed_for(w.index, "rows")).numpy()
+    t0 = time.perf_counter()
+    qr = orope.rope3d(q, grid)[:, sel]
+    kr = orope.rope3d(k, grid)
+    oattn.attention(qr, kr, v, 1.0 / math.sqrt(128))
+    dt = time.perf_counter() - t0
+    flops = 4.0 * len(sel) * L * 128
+    text = ("%d sampled query rows x 1 head x %d keys (RoPE + fp64 softmax "
+            "attention), %s" % (len(sel), L, w.name))
+    return dt, flops, text
+
+
+def run_reference(args, w, rank, world):
+    if rank != 0:
+        return
+    rows = max(16, args.cpu_rows // 32)
+    for _ in range(args.warmup):
+        cpu_oracle_sample(w, rows)
+    total_t, total_f, text = 0.0, 0.0, ""
+    for _ in range(args.steps):
+        dt, fl, text = cpu_oracle_sample(w, rows)
+        total_t += dt
+        total_f += fl
+    tflops = total_f / total_t / 1e12
+    cores = blas_threads()
+    line = {
+        "impl": "reference",
+        "metric": "self-attn TFLOP/s",
+        "value": tflops,
+        "unit": "TFLOP/s",
+        "n_gpus": args.gpus,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": 1e3 * total_t / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": w.name, "sample": text},
+        "cpu_baseline": {"value": tflops, "unit": "TFLOP/s", "cores": cores,
+                         "kind": "oracle", "sample": text},
+        "e2e": {"value": tflops, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------- wan ---
+
+def run_wan(args, w, rank, world, local_rank):
+    import numpy as np
+    import torch
+
+    from video_diffusion_transformer_self_b200 import inputs, wan
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.current_stream()
+
+    lat, g = wan.token_grid(w.frames, w.height, w.width)
+    L = g.F * g.H * g.W
+    B, H = w.batch, w.heads
+    n_lat = int(np.prod(lat)) * B
+    sigmas = wan.fm_sigmas(w.steps, w.shift)
+    seed_off = 7919 * rank  # every rank runs its own independent problem
+
+    def sd(role):
+        return inputs.seed_for(w.index, role) + seed_off
+
+    shape = (B, L, H, 128)
+    ctx_shape = (B, w.text_tokens, H, 128)
+    host = {
+        "q": inputs.randn_bf16(shape, sd("q")),
+        "k": inputs.randn_bf16(shape, sd("k")),
+        "v": inputs.randn_bf16(shape, sd("v")),
+        "k_ctx": inputs.randn_bf16(ctx_shape, sd("k_ctx")),
+        "v_ctx": inputs.randn_bf16(ctx_shape, sd("v_ctx")),
+        "x": inputs.randn_f32((n_lat,), sd("x")),
+        "v_cond": inputs.randn_f32((n_lat,), sd("v_cond")),
+        "v_uncond": inputs.randn_f32((n_lat,), sd("v_uncond")),
+    }
+    lens = inputs.uniform_int(B, w.text_len_lo, w.text_len_hi,
+                              sd("lens")).tolist()
+    d = {kk: t.to(dev) for kk, t in host.items()}
+    o = torch.empty_like(d["q"])
+    oc = torch.empty_like(d["q"])
+    table = wan.rope3d_table(g)
+    guide = 4.0
+    flops_self = 4.0 * B * H * L * L * 128
+
+    ev_pairs = []
+
+    def step(i, timed):
+        s0, s1 = sigmas[i % w.steps], sigmas[i % w.steps + 1]
+        if timed:
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+        if args.rope == "pre":
+            wan.rope3d_qk(d["q"], d["k"], g, table)
+            wan.self_attn(d["q"], d["k"], d["v"], o, g)
+        else:
+            wan.self_attn(d["q"], d["k"], d["v"], o, g, table=table)
+        if timed:
+            e1.record(stream)
+            ev_pairs.append((e0, e1))
+        wan.cross_attn(o, d["k_ctx"], d["v_ctx"], oc, lens)
+        wan.fm_step(d["x"], d["v_cond"], d["v_uncond"], guide, s0, s1)
+
+    launches_per_step = 4 if args.rope == "pre" else 3
+
+    dist = None
+    if world > 1:
+        import torch.distributed as dist_mod
+        dist = dist_mod
+
+    def barrier():
+        if dist is not None:
+            dist.barrier(device_ids=[local_rank])
+
+    for i in range(args.warmup):
+        step(i, False)
+    torch.cuda.synchronize()
+    if wan.device_status() != 0:
+        raise RuntimeError("device timeout during warm-up")
+
+    clocks = ClockSampler(local_rank) if rank == 0 else None
+    barrier()
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(i, True)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop() if clocks else None
+    ms = t_start.elapsed_time(t_end)
+    if wan.device_status() != 0:
+        raise RuntimeError("device timeout during the timed steps")
+    # self-attention kernel time (includes the RoPE pass with --rope pre)
+    attn_ms = [a.elapsed_time(b) for a, b in ev_pairs]
+    attn_avg = sum(attn_ms) / len(attn_ms)
+    if dist is not None:
+        t = torch.tensor([ms, attn_avg], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, attn_avg = float(t[0]), float(t[1])
+
+    # ----- end to end: host buffers in, results out, every step -----
+    e2e = None
+    if not args.no_e2e:
+        pin = {kk: t.pin_memory() for kk, t in host.items()}
+        out_host = torch.empty(oc.shape, dtype=oc.dtype).pin_memory()
+        x_host = torch.empty(n_lat, dtype=torch.float32).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in pin.values())
+        d2h = out_host.numel() * 2 + x_host.numel() * 4
+
+        def e2e_step(i):
+            for kk, t in pin.items():
+                d[kk].copy_(t, non_blocking=True)
+            step(i, False)
+            out_host.copy_(oc, non_blocking=True)
+            x_host.copy_(d["x"], non_blocking=True)
+
+        e2e_step(0)
+        torch.cuda.synchronize()
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(args.steps):
+            e2e_step(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e2e_ms = e0.elapsed_time(e1)
+        if dist is not None:
+            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t[0])
+        e2e = {"value": world * flops_self * args.steps / (e2e_ms / 1e3)
+               / 1e12,
+               "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h,
+               "ms_per_step": e2e_ms / args.steps}
+
+    if rank != 0:
+        return
+    pk, pk_kind = peaks()
+    peak = float(pk.get("bf16_tflops_sustained", 1400.0))
+    value = world * flops_self * args.steps / (ms / 1e3) / 1e12
+    achieved = flops_self / (attn_avg / 1e3) / 1e12
+    line = {
+        "metric": "self-attn TFLOP/s",
+        "value": value,
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {
+            "workload": w.name, "batch": B, "heads": H, "seq_len": L,
+            "grid": [g.F, g.H, g.W], "text_tokens": w.text_tokens,
+            "text_lens": lens, "latent": list(lat), "rope": args.rope,
+            "parallelism": "replicas" if world > 1 else "single",
+            "l2": "inputs larger than L2 (Q/K/V %.0f MB each)"
+                  % (B * L * H * 256 / 1e6),
+        },
+        "frac_of_peak": {
+            "dense_bf16_datasheet_2250": value / 2250.0,
+            "measured_burst": value / float(pk.get("bf16_tflops", 1590.0)),
+            "measured_sustained": value / peak,
+        },
+        "roofline": {
+            "kernel": "self_attn" + ("+rope3d_qk" if args.rope == "pre"
+                                     else " (fused RoPE)"),
+            "bound": "tensor", "achieved": achieved, "peak": peak,
+            "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+            "peak_kind": pk_kind + " sustained bf16 (kernel timed inside a "
+                                   "long step)",
+            "avg_launch_ms": attn_avg,
+        },
+        "gpu_launches": launches_per_step * args.steps,
+        "e2e": e2e,
+        "clocks": clk,
+    }
+    if not args.no_cpu_baseline and world == 1:
+        dt, fl, text = cpu_oracle_sample(w, args.cpu_rows)
+        line["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": "TFLOP/s",
+                                "cores": blas_threads(), "kind": "oracle",
+                                "sample": text, "seconds": dt}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    from video_diffusion_transformer_self_b200.workloads import by_name
+    w = by_name(args.workload)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, w, rank, world)
+        return
+    from video_diffusion_transformer_self_b200 import build
+    if rank == 0 or world == 1:
+        build.build()
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl",
+                                timeout=datetime.timedelta(seconds=120))
+        dist.barrier(device_ids=[local_rank])
+    try:
+        run_wan(args, w, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,159 @@
+/*
+ * wan.h -- C ABI of libwan, the B200 (sm_100a) hot path of the Wan2.1 /
+ * Wan2.2 video diffusion transformer: 3D RoPE, full spatio-temporal
+ * self-attention, length-masked cross-attention to text, and the shifted
+ * sigma schedule with the fused CFG + Euler flow step.
+ *
+ * Sources (cited by page and section):
+ *   "Wan2.2 source reading" -- blog.leeguoo.com, "動画生成の勘定を明らかにする：
+ *       Wan2.2 ソースコード精読";
+ *   "Wan paper explainer"   -- 0h-n0.github.io, "論文解説: Wan - 大規模オープン
+ *       ソース動画生成モデルのアーキテクチャと訓練".
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Attention tensors are bf16, contiguous, row-major [B, L, heads, head_dim]
+ *   (token-major, heads interleaved: the natural layout of a [B, L, dim]
+ *   projection with dim = heads * head_dim).  head_dim must be 128.
+ * - Token order inside L is frame-major: n = (f * H + h) * W + w.
+ * - Device pointers are plain CUDA device addresses owned by the caller; the
+ *   library allocates no device memory and keeps no per-call state.  Every
+ *   launch goes to the caller's stream `s` (a cudaStream_t passed as void*,
+ *   NULL = legacy default stream).  No call synchronises the stream.
+ * - Return values: WAN_OK (0) or a negative wan_status.  Argument checks are
+ *   synchronous and leave the device untouched.  A failed launch returns
+ *   WAN_ECUDA.  Device-side faults surface at the caller's next synchronise.
+ * - Every wait inside a kernel is bounded (about two seconds); a wait that
+ *   runs out records WAN_ETIMEOUT in a device status word, read and cleared
+ *   by wan_device_status().
+ */
+#ifndef WAN_H_
+#define WAN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Token grid after the (1, 2, 2) patchify: L = F * H * W. */
+typedef struct {
+  int32_t F, H, W;
+} wan_grid_t;
+
+enum wan_status {
+  WAN_OK = 0,
+  WAN_EINVAL = -1,        /* bad size, null pointer, out-of-range value   */
+  WAN_EALIGN = -2,        /* pointer not 16-byte aligned                   */
+  WAN_EUNSUPPORTED = -3,  /* current device is not sm_100 (B200 class)     */
+  WAN_ECUDA = -4,         /* a CUDA runtime call or launch failed          */
+  WAN_ETIMEOUT = -5       /* a bounded in-kernel wait ran out              */
+};
+
+/* Static text of a status code (never NULL). */
+const char* wan_status_string(int status);
+
+/* Library ABI version (major * 100 + minor). */
+int wan_version(void);
+
+/* ---------------------------------------------------------------- grid --
+ * Wan2.2 source reading, ch. 2 "VAE" (target_shape, vae_stride (4, 8, 8),
+ * frames of the form 4n+1) and ch. 4 "From latent to token" (patch (1,2,2)).
+ * Host only.  frames = 4n+1 >= 1, height and width multiples of 16 (8 for
+ * the VAE times 2 for the patch).  Writes the latent shape
+ * (16, (frames-1)/4+1, height/8, width/8) to latent_out[4] if it is not NULL
+ * and the token grid to *grid_out.  Returns WAN_EINVAL otherwise.          */
+int wan_token_grid(int frames, int height, int width, int32_t* latent_out,
+                   wan_grid_t* grid_out);
+
+/* ---------------------------------------------------------------- RoPE --
+ * Wan2.2 source reading, ch. 4, section "3D RoPE": per head the 128
+ * channels split into a time band of 44 and height / width bands of 42
+ * (concatenated t, h, w); adjacent channels (2j, 2j+1) form one complex
+ * number that is turned by pos * theta^(-2j / D_band), pos being the
+ * token's f, h or w coordinate; the page rotates in float64.
+ *
+ * Table layout (float2 = {cos, sin}, fp32, computed in fp64 on the host):
+ *   rows 0 .. F-1        : time band,   entry e = j        (j = 0..21)
+ *   rows F .. F+H-1      : height band, entry e = j        (j = 0..20), e=21 pad
+ *   rows F+H .. F+H+W-1  : width band,  entry e = j + 1    (j = 0..20), e=0 pad
+ * every row has 22 entries (176 bytes), pads hold {1, 0}.  With this layout
+ * the absolute pair index p = 2m, 2m+1 of a 16-byte load always lands on a
+ * 16-byte aligned table address.
+ *
+ * wan_rope3d_table_bytes: size of that table.  Returns 0 for a bad grid.
+ * wan_rope3d_table: fills caller-owned device memory d_table (bytes >= the
+ *   size above) with an asynchronous copy from a library-held host staging
+ *   buffer on stream s.  grid sides must be in 1..1024 (the page builds the
+ *   tables for 1024 positions), head_dim 128, theta > 0.  Not capturable in a
+ *   CUDA graph (pageable host copy).
+ * wan_rope3d_qk: rotates q and k in place (bf16 in, fp32 arithmetic, bf16
+ *   out), [B, L, heads, 128] with L = F*H*W, using the table above.  q or k
+ *   may be NULL to rotate only the other.                                   */
+size_t wan_rope3d_table_bytes(wan_grid_t g, int head_dim);
+int wan_rope3d_table(wan_grid_t g, int head_dim, double theta, void* d_table,
+                     size_t bytes, void* s);
+int wan_rope3d_qk(void* q, void* k, int B, wan_grid_t g, int heads,
+                  int head_dim, const void* d_table, void* s);
+
+/* ------------------------------------------------------- self-attention --
+ * Wan2.2 source reading, ch. 4 "Full forward of one block" and ch. 8 "What
+ * is 75600^2": full bidirectional attention over all L = F*H*W tokens,
+ *   O = softmax(Q K^T * softmax_scale) V,   no mask.
+ * q, k, v, o: [B, L, heads, 128] bf16, 16-byte aligned; o must not alias
+ * q, k or v.  If d_table is not NULL (the table above for grid g), Q and K
+ * are rotated by the 3D RoPE inside the kernel as their tiles are staged
+ * (q and k in memory are left untouched); if NULL, q and k are used as given
+ * (already rotated, e.g. by wan_rope3d_qk).  fp32 accumulation and softmax,
+ * bf16 output.  softmax_scale > 0 (the pages use 1/sqrt(head_dim)).        */
+int wan_self_attn(const void* q, const void* k, const void* v, void* o,
+                  int B, wan_grid_t g, int heads, int head_dim,
+                  const void* d_table, float softmax_scale, void* s);
+
+/* ------------------------------------------------------ cross-attention --
+ * Wan2.2 source reading, ch. 3 "Where did the prompt go" (each prompt is
+ * trimmed to its true length; video tokens query, the text context is
+ * key/value) and Wan paper explainer, section "Text encoder"
+ * (softmax(Q K_text^T / sqrt(d_k)) V_text):
+ *   O[b] = softmax(Q[b] K_ctx[b, :len_b]^T * softmax_scale) V_ctx[b, :len_b]
+ * q, o: [B, Lq, heads, 128]; k_ctx, v_ctx: [B, Lk, heads, 128] bf16.
+ * ctx_lens: HOST array of B int32 with 1 <= len_b <= Lk; it is read during
+ * the call.  Rows j >= len_b of k_ctx / v_ctx are never used, whatever they
+ * hold (NaN included).  No RoPE.  B <= 512.                               */
+int wan_cross_attn(const void* q, const void* k_ctx, const void* v_ctx,
+                   void* o, const int32_t* ctx_lens, int B, int Lq, int Lk,
+                   int heads, int head_dim, float softmax_scale, void* s);
+
+/* ------------------------------------------------------------- sampler --
+ * Wan2.2 source reading, ch. 5, section "shift": the points are laid
+ * uniformly and mapped by sigma = shift*s / (1 + (shift-1)*s); ch. 1
+ * "One ruler, two scales": t = 1000 * sigma.
+ * wan_fm_sigmas: host, fp64.  Writes sigma_0 .. sigma_N (n_steps + 1
+ *   values) to sigmas_out with s_i = s_max * (1 - i/n_steps), i < n_steps,
+ *   and sigma_N = 0.  n_steps >= 1, shift > 0, 0 < s_max <= 1.
+ *
+ * Wan2.2 source reading, ch. 5 "UniPC" (Euler: velocity held constant over
+ * the step) and "CFG" (uncond + w * (cond - uncond)):
+ * wan_fm_step: x[i] += (sigma_next - sigma) * v[i], with
+ *   v = v_cond                                   if v_uncond == NULL,
+ *   v = v_uncond + guide * (v_cond - v_uncond)   otherwise,
+ *   all fp32 on the device, n elements, in place on x.  dt = sigma_next -
+ *   sigma is formed in fp64 on the host and rounded once to fp32.  x, v_cond
+ *   and v_uncond must be 16-byte aligned; x may not alias the velocities.  */
+int wan_fm_sigmas(int n_steps, double shift, double s_max,
+                  double* sigmas_out);
+int wan_fm_step(float* x, const float* v_cond, const float* v_uncond,
+                float guide, int64_t n, double sigma, double sigma_next,
+                void* s);
+
+/* ------------------------------------------------------------- status ---
+ * Reads (and, if clear != 0, resets) the device status word of the current
+ * device: 0 or WAN_ETIMEOUT.  Synchronous (waits for the device).          */
+int wan_device_status(int clear);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WAN_H_ */

@@ -1,0 +1,206 @@
+"""ctypes binding of libwan.so (declared in include/wan.h).
+
+Argument marshalling only: torch tensors are turned into raw device
+pointers, sizes and the current CUDA stream, and every status code other
+than WAN_OK raises ``WanError``.  All arithmetic of the hot path runs in the
+library's CUDA kernels (or, for the grid / schedule / RoPE-table set-up
+calls, in the library's host code).  There is no fallback: if libwan.so is
+missing or fails to load, importing the functions raises.
+"""
+
+import ctypes
+import math
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libwan.so")
+
+WAN_OK = 0
+WAN_EINVAL = -1
+WAN_EALIGN = -2
+WAN_EUNSUPPORTED = -3
+WAN_ECUDA = -4
+WAN_ETIMEOUT = -5
+
+
+class WanError(RuntimeError):
+    def __init__(self, status, what):
+        self.status = status
+        super().__init__("%s: %s (%d)" % (what, status_string(status), status))
+
+
+class Grid(ctypes.Structure):
+    _fields_ = [("F", ctypes.c_int32), ("H", ctypes.c_int32),
+                ("W", ctypes.c_int32)]
+
+    def __iter__(self):
+        return iter((self.F, self.H, self.W))
+
+    def __repr__(self):
+        return "Grid(%d, %d, %d)" % (self.F, self.H, self.W)
+
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_SIGNATURES = {
+    "wan_status_string": (ctypes.c_char_p, [_I]),
+    "wan_version": (_I, []),
+    "wan_token_grid": (_I, [_I, _I, _I, ctypes.POINTER(ctypes.c_int32),
+                            ctypes.POINTER(Grid)]),
+    "wan_rope3d_table_bytes": (ctypes.c_size_t, [Grid, _I]),
+    "wan_rope3d_table": (_I, [Grid, _I, ctypes.c_double, _P,
+                              ctypes.c_size_t, _P]),
+    "wan_rope3d_qk": (_I, [_P, _P, _I, Grid, _I, _I, _P, _P]),
+    "wan_self_attn": (_I, [_P, _P, _P, _P, _I, Grid, _I, _I, _P,
+                           ctypes.c_float, _P]),
+    "wan_cross_attn": (_I, [_P, _P, _P, _P, ctypes.POINTER(ctypes.c_int32),
+                            _I, _I, _I, _I, _I, ctypes.c_float, _P]),
+    "wan_fm_sigmas": (_I, [_I, ctypes.c_double, ctypes.c_double,
+                           ctypes.POINTER(ctypes.c_double)]),
+    "wan_fm_step": (_I, [_P, _P, _P, ctypes.c_float, ctypes.c_int64,
+                         ctypes.c_double, ctypes.c_double, _P]),
+    "wan_device_status": (_I, [_I]),
+}
+
+_lib = None
+
+
+def lib():
+    """The loaded library (ctypes.CDLL); raises if it cannot be loaded."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                "libwan.so not built: run `python -m "
+                "video_diffusion_transformer_self_b200.build`")
+        l = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGNATURES.items():
+            fn = getattr(l, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = l
+    return _lib
+
+
+def status_string(status):
+    return lib().wan_status_string(int(status)).decode()
+
+
+def _check(status, what):
+    if status != WAN_OK:
+        raise WanError(status, what)
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _bf16_bl(t, name):
+    import torch
+    if t.dtype != torch.bfloat16 or t.dim() != 4 or not t.is_contiguous() \
+            or not t.is_cuda:
+        raise ValueError("%s must be a contiguous CUDA bf16 [B, L, heads, d]"
+                         " tensor" % name)
+
+
+# ---------------------------------------------------------------- host ---
+
+def token_grid(frames, height, width):
+    """(latent shape (16, F, h, w), token Grid) for a pixel video."""
+    lat = (ctypes.c_int32 * 4)()
+    g = Grid()
+    _check(lib().wan_token_grid(frames, height, width, lat, ctypes.byref(g)),
+           "wan_token_grid")
+    return tuple(lat), g
+
+
+def grid(F, H, W):
+    return Grid(F, H, W)
+
+
+def fm_sigmas(n_steps, shift, s_max=1.0):
+    """sigma_0 .. sigma_N (list of N + 1 floats)."""
+    out = (ctypes.c_double * (n_steps + 1))()
+    _check(lib().wan_fm_sigmas(n_steps, shift, s_max, out), "wan_fm_sigmas")
+    return list(out)
+
+
+def rope3d_table_bytes(g, head_dim=128):
+    return lib().wan_rope3d_table_bytes(g, head_dim)
+
+
+# -------------------------------------------------------------- device ---
+
+def rope3d_table(g, theta=10000.0, head_dim=128, out=None, stream=None):
+    """Device RoPE table for grid g (a uint8 CUDA tensor)."""
+    import torch
+    n = rope3d_table_bytes(g, head_dim)
+    if n == 0:
+        raise WanError(WAN_EINVAL, "wan_rope3d_table_bytes")
+    if out is None:
+        out = torch.empty(n, dtype=torch.uint8, device="cuda")
+    _check(lib().wan_rope3d_table(g, head_dim, theta, _ptr(out), out.numel(),
+                                  _stream(stream)), "wan_rope3d_table")
+    return out
+
+
+def rope3d_qk(q, k, g, table, stream=None):
+    """In-place 3D RoPE of q and k ([B, L, heads, 128] bf16)."""
+    t = q if q is not None else k
+    _bf16_bl(t, "q/k")
+    _check(lib().wan_rope3d_qk(_ptr(q), _ptr(k), t.shape[0], g, t.shape[2],
+                               t.shape[3], _ptr(table), _stream(stream)),
+           "wan_rope3d_qk")
+
+
+def self_attn(q, k, v, o, g, table=None, softmax_scale=None, stream=None):
+    """o = softmax(rope(q) rope(k)^T * scale) v; RoPE fused if table given."""
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o)):
+        _bf16_bl(t, name)
+    B, L, H, D = q.shape
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(D)
+    _check(lib().wan_self_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, g, H, D,
+                               _ptr(table), softmax_scale, _stream(stream)),
+           "wan_self_attn")
+
+
+def cross_attn(q, k_ctx, v_ctx, o, ctx_lens, softmax_scale=None,
+               stream=None):
+    """o[b] = softmax(q[b] k_ctx[b,:len_b]^T * scale) v_ctx[b,:len_b]."""
+    for name, t in (("q", q), ("k_ctx", k_ctx), ("v_ctx", v_ctx), ("o", o)):
+        _bf16_bl(t, name)
+    B, Lq, H, D = q.shape
+    Lk = k_ctx.shape[1]
+    lens = (ctypes.c_int32 * B)(*[int(x) for x in ctx_lens])
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(D)
+    _check(lib().wan_cross_attn(_ptr(q), _ptr(k_ctx), _ptr(v_ctx), _ptr(o),
+                                lens, B, Lq, Lk, H, D, softmax_scale,
+                                _stream(stream)), "wan_cross_attn")
+
+
+def fm_step(x, v_cond, v_uncond, guide, sigma, sigma_next, stream=None):
+    """x += (sigma_next - sigma) * (v_uncond + guide (v_cond - v_uncond))."""
+    import torch
+    for t in (x, v_cond) + ((v_uncond,) if v_uncond is not None else ()):
+        if t.dtype != torch.float32 or not t.is_contiguous() or not t.is_cuda:
+            raise ValueError("fm_step tensors must be contiguous CUDA fp32")
+    _check(lib().wan_fm_step(_ptr(x), _ptr(v_cond), _ptr(v_uncond), guide,
+                             x.numel(), sigma, sigma_next, _stream(stream)),
+           "wan_fm_step")
+
+
+def device_status(clear=True):
+    """0, or WAN_ETIMEOUT if a bounded in-kernel wait ran out."""
+    st = lib().wan_device_status(1 if clear else 0)
+    if st not in (0, WAN_ETIMEOUT):
+        _check(st, "wan_device_status")
+    return st
