@@ -9,24 +9,28 @@
 // prompt's true length take no part.  Wan paper explainer, section "Text
 // encoder": softmax(Q K_text^T / sqrt(d_k)) V_text.
 //
-// One CTA per (128-row query tile, head, batch row).  Warp roles:
-//   warps 0-3  softmax: thread r owns query row r (TMEM lane r); reads a
-//              128x128 fp32 score tile from TMEM, keeps the running row max
-//              and sum, writes P (bf16) back into TMEM over the scores it
-//              came from, rescales the O accumulator in TMEM when the max
-//              grows by more than 2^8, and runs the epilogue (O / l -> bf16).
-//   warp 4     TMA producer: Q tile once, then K / V tiles through an
-//              NS-stage ring.
-//   warp 5     MMA issuer (one elected lane): S = Q K^T (SS form, both
-//              operands K-major in smem) into one of two TMEM score buffers,
-//              O += P V (TS form, P from TMEM, V MN-major in smem).
-//   warps 6-7  (RoPE variant only) rotate the Q tile and every K tile in
-//              shared memory before the tensor cores read them (two rows
-//              per thread; 8 warps keep the 255-register cap per thread).
-// Tensor memory: columns [0,128) and [128,256) score / P buffers (double
-// buffered so S(j+1) runs while row j's softmax works), [256,384) O.
-// Tiles are stored as two 64-column halves, each [128 rows][128 B] with the
-// 128-byte swizzle TMA writes and UMMA reads.
+// One CTA per (256 query rows = two 128-row tiles, head, batch row).  The two
+// tiles ping-pong: while the softmax of one tile runs, the tensor cores run
+// the other tile's P V and next Q K^T, so neither waits on the other.
+// Warp roles (384 threads, registers rebalanced with setmaxnreg):
+//   warps 0-3 / 4-7  softmax of tile 0 / tile 1: thread r owns query row r
+//              (TMEM lane r).  Reads the 128x128 fp32 score tile from TMEM,
+//              keeps the running row max (log2 units) and sum, writes P
+//              (bf16) back into TMEM over its scores, rescales O in TMEM when
+//              the max grows by more than 2^8 (exact after the final O / l),
+//              and writes the bf16 epilogue.  A quarter of the exponentials
+//              run on the FMA pipe (exp2_fma2) to offload the MUFU unit.
+//   warp 8     TMA producer: the two Q tiles once, then K (3-stage ring) and
+//              V (2-stage ring).
+//   warp 9     MMA issuer (one lane): S_t = Q_t K^T (both operands K-major in
+//              smem) and O_t += P_t V (P from TMEM, V MN-major in smem), in
+//              the order PV_0(j-1), S_0(j), PV_1(j-1), S_1(j).
+//   warps 10-11  RoPE variant: rotate the Q tiles and every K tile in shared
+//              memory before the tensor cores read them.
+// Tensor memory (512 columns): S/P of tile 0 at 0, of tile 1 at 128, O of
+// tile 0 at 256, of tile 1 at 384.  Operand tiles are [128 rows][128 ch]
+// bf16 stored as two 64-channel halves of [128][128 B] with the 128-byte
+// swizzle that TMA writes and UMMA reads.
 #include <math.h>
 
 #include <mutex>
@@ -40,17 +44,24 @@ __device__ int g_wan_status = 0;
 namespace {
 
 constexpr int BM = 128;                      // query rows per tile
+constexpr int QT = 2;                        // query tiles per CTA
 constexpr int BN = 128;                      // keys per block
 constexpr int HD = 128;                      // head dim
-constexpr int NS = 3;                        // K / V ring stages
+constexpr int NSK = 3;                       // K ring stages
+constexpr int NSV = 2;                       // V ring stages
 constexpr uint32_t HALF = 16384;             // one [128][64] bf16 half tile
 constexpr uint32_t TILE = 2 * HALF;          // one [128][128] bf16 tile
-constexpr uint32_t SMEM_DYN = TILE * (1 + 2 * NS) + 1024;
+constexpr uint32_t SMEM_DYN = TILE * (QT + NSK + NSV) + 1024;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t TM_O = 256;               // O accumulator column
+constexpr uint32_t TM_O = 256;               // O of tile t at TM_O + 128 t
+constexpr int kThreads = 384;
+constexpr int kSoftmaxRegs = 216;            // warps 0-7
+constexpr int kOtherRegs = 72;               // warps 8-11
+constexpr int kRopeThreads = 64;             // warps 10-11
 constexpr int MAX_CROSS_BATCH = 512;
-constexpr int kRopeThreads = 64;             // warps 6-7 of the RoPE variant
 constexpr float RESCALE_LOG2 = 8.0f;         // rescale O when max grows > 2^8
+// Pairs (2e, 2e+1) with (e & 7) < kEmuPer8 take the FMA-pipe exponential.
+constexpr int kEmuPer8 = 2;
 
 constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, BN, 0);   // K-major B
 constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, HD, 1);  // MN-major B
@@ -70,23 +81,89 @@ enum : int {
   B_QFULL = 0,
   B_QREADY = 1,
   B_KFULL = 2,
-  B_KREADY = B_KFULL + NS,
-  B_VFULL = B_KREADY + NS,
-  B_KEMPTY = B_VFULL + NS,
-  B_VEMPTY = B_KEMPTY + NS,
-  B_SFULL = B_VEMPTY + NS,  // 2
-  B_PFULL = B_SFULL + 2,    // 2
-  B_ODONE = B_PFULL + 2,
-  B_OFINAL = B_ODONE + 1,   // the last PV only (single phase)
-  B_DRAIN = B_OFINAL + 1,
+  B_KREADY = B_KFULL + NSK,
+  B_KEMPTY = B_KREADY + NSK,
+  B_VFULL = B_KEMPTY + NSK,
+  B_VEMPTY = B_VFULL + NSV,
+  B_SFULL = B_VEMPTY + NSV,  // per tile
+  B_PFULL = B_SFULL + QT,    // per tile, one arrival per softmax warp
+  B_OFINAL = B_PFULL + QT,   // per tile, the last PV only (single phase)
+  B_DRAIN = B_OFINAL + QT,
   NBAR = B_DRAIN + 1
 };
+
+// ------------------------------------------------------- small helpers --
 
 __device__ __forceinline__ float2 bf16x2_to_float2(uint32_t v) {
   float2 r;
   r.x = __uint_as_float(v << 16);
   r.y = __uint_as_float(v & 0xFFFF0000u);
   return r;
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+__device__ __forceinline__ float2 fsub2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "sub.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+// 2^x for two lanes on the FMA pipe.  Cody-Waite style reduction
+// x = n + f, n = round-to-nearest(x) by the 1.5 * 2^23 add (n lands in the
+// low mantissa bits of j), f in [-0.5, 0.5]; 2^f by a degree-3 polynomial
+// fitted here (csrc/fit_exp2.py: weighted least squares on Chebyshev nodes,
+// max relative error 1.2e-4 on [-126, 8]); 2^n applied by adding n << 23 to
+// the bit pattern.  x is clamped to >= -126 so the exponent cannot wrap.
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+  x.x = fmaxf(x.x, -126.0f);
+  x.y = fmaxf(x.y, -126.0f);
+  const float2 magic = make_float2(12582912.0f, 12582912.0f);
+  const float2 j = fadd2(x, magic);
+  const float2 f = fsub2(x, fsub2(j, magic));
+  float2 p = ffma2(make_float2(5.459282547e-02f, 5.459282547e-02f), f,
+                   make_float2(2.422178388e-01f, 2.422178388e-01f));
+  p = ffma2(p, f, make_float2(6.933686137e-01f, 6.933686137e-01f));
+  p = ffma2(p, f, make_float2(1.0f, 1.0f));
+  return make_float2(
+      __uint_as_float(__float_as_uint(p.x) + (__float_as_uint(j.x) << 23)),
+      __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(j.y) << 23)));
+}
+
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
+}
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kOtherRegs));
 }
 
 // Rotate row r of a swizzled [128][128] bf16 tile in shared memory by the
@@ -135,8 +212,56 @@ __device__ __forceinline__ void rope_row(uint8_t* tile, int r, int n,
   }
 }
 
+// Row max of 128 scores with 3-input max and four independent chains.
+__device__ __forceinline__ float rowmax128(const float* s) {
+  float m0 = s[0], m1 = s[1], m2 = s[2], m3 = s[3];
+#pragma unroll
+  for (int c = 4; c < BN; c += 8) {
+    m0 = fmax3(m0, s[c + 0], s[c + 1]);
+    m1 = fmax3(m1, s[c + 2], s[c + 3]);
+    m2 = fmax3(m2, s[c + 4], s[c + 5]);
+    m3 = fmax3(m3, s[c + 6], s[c + 7]);
+  }
+  return fmaxf(fmax3(m0, m1, m2), m3);
+}
+
+// p = 2^(s * c2 - m) for 128 scores, packed bf16 P stored into TMEM at
+// `pcol` (64 columns), sum of p returned.  kEmu: use the FMA-pipe
+// exponential for part of the pairs (never for a masked block, whose -inf
+// entries must give exact zeros).
+template <bool kEmu>
+__device__ __forceinline__ float exp_store_row(const float* s, float c2,
+                                               float m, uint32_t pcol) {
+  const float2 c22 = make_float2(c2, c2);
+  const float2 nm2 = make_float2(-m, -m);
+  float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                   make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const int pair = c * 16 + e;
+      const float2 x =
+          ffma2(make_float2(s[2 * pair], s[2 * pair + 1]), c22, nm2);
+      float2 p;
+      if (kEmu && (pair & 7) < kEmuPer8) {
+        p = exp2_fma2(x);
+      } else {
+        p.x = ex2(x.x);
+        p.y = ex2(x.y);
+      }
+      acc[e & 3] = fadd2(acc[e & 3], p);
+      pk[e] = pack_bf16x2(p.x, p.y);
+    }
+    tmem_st16(pcol + c * 16, pk);
+  }
+  const float2 t = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
+  return t.x + t.y;
+}
+
 template <int kRope>
-__global__ void __launch_bounds__(kRope ? 256 : 192, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v,
@@ -148,7 +273,7 @@ __global__ void __launch_bounds__(kRope ? 256 : 192, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int q0 = blockIdx.x * BM;
+  const int q0 = blockIdx.x * (QT * BM);
   const int head = blockIdx.y;
   const int b = blockIdx.z;
   const int kv_len = args.cross ? args.lens[b] : args.Lk;
@@ -158,175 +283,246 @@ __global__ void __launch_bounds__(kRope ? 256 : 192, 1)
 
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* sm = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-  uint8_t* sQ = sm;
-  uint8_t* sK = sm + TILE;
-  uint8_t* sV = sK + NS * TILE;
+  uint8_t* sQ = sm;                   // QT tiles
+  uint8_t* sK = sm + QT * TILE;       // NSK tiles
+  uint8_t* sV = sK + NSK * TILE;      // NSV tiles
 
   if (threadIdx.x == 0) {
     s_abort = 0;
     mbar_init(&bar[B_QFULL], 1);
     mbar_init(&bar[B_QREADY], kRopeThreads);
-    for (int i = 0; i < NS; ++i) {
+    for (int i = 0; i < NSK; ++i) {
       mbar_init(&bar[B_KFULL + i], 1);
       mbar_init(&bar[B_KREADY + i], kRopeThreads);
-      mbar_init(&bar[B_VFULL + i], 1);
       mbar_init(&bar[B_KEMPTY + i], 1);
+    }
+    for (int i = 0; i < NSV; ++i) {
+      mbar_init(&bar[B_VFULL + i], 1);
       mbar_init(&bar[B_VEMPTY + i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&bar[B_SFULL + i], 1);
-      mbar_init(&bar[B_PFULL + i], 4);
+    for (int t = 0; t < QT; ++t) {
+      mbar_init(&bar[B_SFULL + t], 1);
+      mbar_init(&bar[B_PFULL + t], 4);
+      mbar_init(&bar[B_OFINAL + t], 1);
     }
-    mbar_init(&bar[B_ODONE], 1);
-    mbar_init(&bar[B_OFINAL], 1);
     mbar_init(&bar[B_DRAIN], 1);
     fence_mbar_init();
   }
-  if (warp == 5) tmem_alloc(&s_tmem, TMEM_COLS);
+  if (warp == 9) tmem_alloc(&s_tmem, TMEM_COLS);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s_tmem;
 
-  if (warp == 4) {
-    // ------------------------------------------------------ TMA producer --
-    if (lane == 0) {
-      prefetch_tmap(&tm_q);
-      prefetch_tmap(&tm_k);
-      prefetch_tmap(&tm_v);
-    }
-    bool ok = true;
-    int nk = 0, nv = 0;  // K / V tiles issued
-    if (lane == 0) {
-      mbar_expect_tx(&bar[B_QFULL], TILE);
-      tma_load_4d(sQ, &tm_q, &bar[B_QFULL], 0, head, q0, b);
-      tma_load_4d(sQ + HALF, &tm_q, &bar[B_QFULL], 64, head, q0, b);
-    }
-    for (int j = 0; j < nblk && ok; ++j) {
-      const int st = j % NS;
-      const int use = j / NS;
-      if (use > 0) ok = wait_warp(&bar[B_KEMPTY + st], (use - 1) & 1,
-                                  abort_flag, status);
-      if (!ok) break;
+  if (warp >= 8) {
+    // Warpgroup 2: producer, MMA issuer, RoPE.  Registers handed to the
+    // softmax warpgroups first (setmaxnreg must open the warpgroup's branch).
+    setmaxnreg_dec();
+    if (warp == 8) {
+      // ------------------------------------------------------ TMA producer --
       if (lane == 0) {
-        mbar_expect_tx(&bar[B_KFULL + st], TILE);
-        tma_load_4d(sK + st * TILE, &tm_k, &bar[B_KFULL + st], 0, head,
-                    j * BN, b);
-        tma_load_4d(sK + st * TILE + HALF, &tm_k, &bar[B_KFULL + st], 64,
-                    head, j * BN, b);
-      }
-      ++nk;
-      if (use > 0) ok = wait_warp(&bar[B_VEMPTY + st], (use - 1) & 1,
-                                  abort_flag, status);
-      if (!ok) break;
-      if (lane == 0) {
-        mbar_expect_tx(&bar[B_VFULL + st], TILE);
-        tma_load_4d(sV + st * TILE, &tm_v, &bar[B_VFULL + st], 0, head,
-                    j * BN, b);
-        tma_load_4d(sV + st * TILE + HALF, &tm_v, &bar[B_VFULL + st], 64,
-                    head, j * BN, b);
-      }
-      ++nv;
-      __syncwarp();
-    }
-    if (*abort_flag) {
-      // Let copies already issued land before the CTA leaves.
-      wait_warp_drain(&bar[B_QFULL], 0, status);
-      for (int j = (nk > NS ? nk - NS : 0); j < nk; ++j)
-        wait_warp_drain(&bar[B_KFULL + j % NS], (j / NS) & 1, status);
-      for (int j = (nv > NS ? nv - NS : 0); j < nv; ++j)
-        wait_warp_drain(&bar[B_VFULL + j % NS], (j / NS) & 1, status);
-    }
-  } else if (warp == 5) {
-    // -------------------------------------------------------- MMA issuer --
-    const uint32_t sQa = smem_u32(sQ);
-    const uint32_t sKa = smem_u32(sK);
-    const uint32_t sVa = smem_u32(sV);
-    bool ok = wait_warp(&bar[kRope ? B_QREADY : B_QFULL], 0, abort_flag,
-                        status);
-    auto issue_pv = [&](int i) -> bool {
-      const int pb = i & 1;
-      const int st = i % NS;
-      if (!wait_warp(&bar[B_PFULL + pb], (i >> 1) & 1, abort_flag, status))
-        return false;
-      if (!wait_warp(&bar[B_VFULL + st], (i / NS) & 1, abort_flag, status))
-        return false;
-      if (args.cross && kv_len < (i + 1) * BN) {
-        // Text padding rows may hold anything (NaN included): P is 0 there
-        // but 0 * NaN is not, so clear those V rows before the MMA.
-        const int first = kv_len - i * BN;
-        uint8_t* vt = sV + st * TILE;
-        for (int idx = lane; idx < (BN - first) * 16; idx += 32) {
-          const int r = first + (idx >> 4);
-          const int c = idx & 15;
-          *reinterpret_cast<uint4*>(vt + (c >> 3) * HALF + r * 128 +
-                                    ((c & 7) << 4)) = make_uint4(0, 0, 0, 0);
+        prefetch_tmap(&tm_q);
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_v);
+        mbar_expect_tx(&bar[B_QFULL], QT * TILE);
+        for (int t = 0; t < QT; ++t) {
+          tma_load_4d(sQ + t * TILE, &tm_q, &bar[B_QFULL], 0, head,
+                      q0 + t * BM, b);
+          tma_load_4d(sQ + t * TILE + HALF, &tm_q, &bar[B_QFULL], 64, head,
+                      q0 + t * BM, b);
         }
-        fence_proxy_async_smem();
+      }
+      bool ok = true;
+      int nk = 0, nv = 0;  // K / V tiles issued
+      for (int j = 0; j < nblk && ok; ++j) {
+        const int sk = j % NSK, uk = j / NSK;
+        if (uk > 0)
+          ok = wait_warp(&bar[B_KEMPTY + sk], (uk - 1) & 1, abort_flag, status);
+        if (!ok) break;
+        if (lane == 0) {
+          mbar_expect_tx(&bar[B_KFULL + sk], TILE);
+          tma_load_4d(sK + sk * TILE, &tm_k, &bar[B_KFULL + sk], 0, head,
+                      j * BN, b);
+          tma_load_4d(sK + sk * TILE + HALF, &tm_k, &bar[B_KFULL + sk], 64,
+                      head, j * BN, b);
+        }
+        ++nk;
+        const int sv = j % NSV, uv = j / NSV;
+        if (uv > 0)
+          ok = wait_warp(&bar[B_VEMPTY + sv], (uv - 1) & 1, abort_flag, status);
+        if (!ok) break;
+        if (lane == 0) {
+          mbar_expect_tx(&bar[B_VFULL + sv], TILE);
+          tma_load_4d(sV + sv * TILE, &tm_v, &bar[B_VFULL + sv], 0, head,
+                      j * BN, b);
+          tma_load_4d(sV + sv * TILE + HALF, &tm_v, &bar[B_VFULL + sv], 64,
+                      head, j * BN, b);
+        }
+        ++nv;
         __syncwarp();
       }
-      tc_fence_after();
-      if (lane == 0) {
-#pragma unroll
+      if (*abort_flag) {
+        // Let copies already issued land before the CTA leaves.
+        wait_warp_drain(&bar[B_QFULL], 0, status);
+        for (int j = (nk > NSK ? nk - NSK : 0); j < nk; ++j)
+          wait_warp_drain(&bar[B_KFULL + j % NSK], (j / NSK) & 1, status);
+        for (int j = (nv > NSV ? nv - NSV : 0); j < nv; ++j)
+          wait_warp_drain(&bar[B_VFULL + j % NSV], (j / NSV) & 1, status);
+      }
+    } else if (warp == 9) {
+      // -------------------------------------------------------- MMA issuer --
+      const uint32_t sQa = smem_u32(sQ);
+      const uint32_t sKa = smem_u32(sK);
+      const uint32_t sVa = smem_u32(sV);
+      // S_t(j) = Q_t K(j)^T into the score buffer of tile t.
+      auto issue_s = [&](int t, int j) {
+        const int sk = j % NSK;
+  #pragma unroll
+        for (int k = 0; k < HD / 16; ++k) {
+          // K-major operands: 16-channel K slices are 32 B apart inside a
+          // 128-B swizzle row; the second 64-channel half starts 16 KB on.
+          const uint32_t off = (k >> 2) * HALF + (k & 3) * 32;
+          const uint64_t adesc = sdesc_sw128(sQa + t * TILE + off, 16, 1024);
+          const uint64_t bdesc = sdesc_sw128(sKa + sk * TILE + off, 16, 1024);
+          umma_ss(tmem + t * 128, adesc, bdesc, IDESC_S, k > 0 ? 1u : 0u);
+        }
+        umma_commit(&bar[B_SFULL + t]);
+      };
+      // O_t += P_t(i) V(i).
+      auto issue_pv = [&](int t, int i) {
+        const int sv = i % NSV;
+  #pragma unroll
         for (int k = 0; k < BN / 16; ++k) {
           // B = V[16k .. 16k+15][0..127]: MN-major, 8-key groups 1024 B
-          // apart (SBO), the two 64-column halves 16 KB apart (LBO).
+          // apart (SBO), the two 64-channel halves 16 KB apart (LBO).
           const uint64_t bdesc =
-              sdesc_sw128(sVa + st * TILE + k * 2048, HALF, 1024);
-          umma_ts(tmem + TM_O, tmem + pb * 128 + k * 8, bdesc, IDESC_PV,
-                  (i > 0 || k > 0) ? 1u : 0u);
+              sdesc_sw128(sVa + sv * TILE + k * 2048, HALF, 1024);
+          umma_ts(tmem + TM_O + t * 128, tmem + t * 128 + k * 8, bdesc,
+                  IDESC_PV, (i > 0 || k > 0) ? 1u : 0u);
         }
-        umma_commit(&bar[B_ODONE]);
-        umma_commit(&bar[B_VEMPTY + st]);
-        if (i == nblk - 1) umma_commit(&bar[B_OFINAL]);
-      }
-      __syncwarp();
-      return true;
-    };
-    for (int j = 0; j < nblk && ok; ++j) {
-      const int st = j % NS;
-      ok = wait_warp(&bar[(kRope ? B_KREADY : B_KFULL) + st], (j / NS) & 1,
-                     abort_flag, status);
-      if (!ok) break;
-      tc_fence_after();
-      if (lane == 0) {
-        const uint32_t sbuf = tmem + (j & 1) * 128;
-#pragma unroll
-        for (int k = 0; k < HD / 16; ++k) {
-          // K-major operands: 16-element K slices are 32 B apart inside a
-          // 128-B swizzle row; the second 64-column half starts 16 KB on.
-          const uint32_t off = (k >> 2) * HALF + (k & 3) * 32;
-          const uint64_t adesc = sdesc_sw128(sQa + off, 16, 1024);
-          const uint64_t bdesc = sdesc_sw128(sKa + st * TILE + off, 16, 1024);
-          umma_ss(sbuf, adesc, bdesc, IDESC_S, k > 0 ? 1u : 0u);
+      };
+      // Waits for P_0(i) and V(i), clears text-padding rows of V(i).
+      auto ready_pv0 = [&](int i) -> bool {
+        if (!wait_warp(&bar[B_PFULL + 0], i & 1, abort_flag, status))
+          return false;
+        if (!wait_warp(&bar[B_VFULL + i % NSV], (i / NSV) & 1, abort_flag,
+                       status))
+          return false;
+        if (args.cross && kv_len < (i + 1) * BN) {
+          // Text padding rows may hold anything (NaN included): P is 0 there
+          // but 0 * NaN is not, so clear those V rows before the MMA.
+          const int first = kv_len - i * BN;
+          uint8_t* vt = sV + (i % NSV) * TILE;
+          for (int idx = lane; idx < (BN - first) * 16; idx += 32) {
+            const int r = first + (idx >> 4);
+            const int c = idx & 15;
+            *reinterpret_cast<uint4*>(vt + (c >> 3) * HALF + r * 128 +
+                                      ((c & 7) << 4)) = make_uint4(0, 0, 0, 0);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
         }
-        umma_commit(&bar[B_SFULL + (j & 1)]);
-        umma_commit(&bar[B_KEMPTY + st]);
+        tc_fence_after();
+        return true;
+      };
+      bool ok = wait_warp(&bar[kRope ? B_QREADY : B_QFULL], 0, abort_flag,
+                          status);
+      for (int j = 0; j < nblk && ok; ++j) {
+        const int sk = j % NSK;
+        if (j > 0) {
+          ok = ready_pv0(j - 1);
+          if (!ok) break;
+          if (lane == 0) issue_pv(0, j - 1);
+          __syncwarp();
+        }
+        ok = wait_warp(&bar[(kRope ? B_KREADY : B_KFULL) + sk], (j / NSK) & 1,
+                       abort_flag, status);
+        if (!ok) break;
+        tc_fence_after();
+        if (lane == 0) issue_s(0, j);
+        __syncwarp();
+        if (j > 0) {
+          ok = wait_warp(&bar[B_PFULL + 1], (j - 1) & 1, abort_flag, status);
+          if (!ok) break;
+          tc_fence_after();
+          if (lane == 0) {
+            issue_pv(1, j - 1);
+            umma_commit(&bar[B_VEMPTY + (j - 1) % NSV]);
+          }
+          __syncwarp();
+        }
+        if (lane == 0) {
+          issue_s(1, j);
+          umma_commit(&bar[B_KEMPTY + sk]);
+        }
+        __syncwarp();
       }
+      if (ok) {
+        const int i = nblk - 1;
+        ok = ready_pv0(i);
+        if (ok && lane == 0) {
+          issue_pv(0, i);
+          umma_commit(&bar[B_OFINAL + 0]);
+        }
+        __syncwarp();
+        if (ok) ok = wait_warp(&bar[B_PFULL + 1], i & 1, abort_flag, status);
+        if (ok) {
+          tc_fence_after();
+          if (lane == 0) {
+            issue_pv(1, i);
+            umma_commit(&bar[B_OFINAL + 1]);
+            umma_commit(&bar[B_VEMPTY + i % NSV]);
+          }
+        }
+        __syncwarp();
+      }
+      // Drain every MMA before tensor memory is released.
+      if (lane == 0) umma_commit(&bar[B_DRAIN]);
       __syncwarp();
-      if (j >= 1) ok = issue_pv(j - 1);
+      wait_warp_drain(&bar[B_DRAIN], 0, status);
+    } else if (kRope) {
+      // -------------------------------------------------------------- RoPE --
+      const int tr = threadIdx.x - 320;  // 0..63
+      bool ok = wait_warp(&bar[B_QFULL], 0, abort_flag, status);
+      if (ok) {
+        for (int rr = tr; rr < QT * BM; rr += kRopeThreads) {
+          const int n = q0 + rr;
+          if (n < args.Lq) rope_row(sQ + (rr >> 7) * TILE, rr & 127, n, args);
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&bar[B_QREADY]);
+      }
+      for (int j = 0; j < nblk && ok; ++j) {
+        const int sk = j % NSK;
+        ok = wait_warp(&bar[B_KFULL + sk], (j / NSK) & 1, abort_flag, status);
+        if (!ok) break;
+        for (int rr = tr; rr < BN; rr += kRopeThreads)
+          if (j * BN + rr < kv_len)
+            rope_row(sK + sk * TILE, rr, j * BN + rr, args);
+        fence_proxy_async_smem();
+        mbar_arrive(&bar[B_KREADY + sk]);
+      }
     }
-    if (ok) ok = issue_pv(nblk - 1);
-    // Drain every MMA before tensor memory is released.
-    if (lane == 0) umma_commit(&bar[B_DRAIN]);
-    __syncwarp();
-    wait_warp_drain(&bar[B_DRAIN], 0, status);
-  } else if (warp < 4) {
+  } else {
     // ----------------------------------------------------------- softmax --
-    const int r = threadIdx.x;  // query row in the tile == TMEM lane
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    setmaxnreg_inc();
+    const int t = warp >> 2;                 // query tile of this warpgroup
+    const int r = threadIdx.x & 127;         // row in the tile == TMEM lane
+    const uint32_t lane_base =
+        tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const uint32_t s_col = lane_base + t * 128;
+    const uint32_t o_col = lane_base + TM_O + t * 128;
     const float c2 = args.scale_log2;
     float m_run = -INFINITY;
     float l_run = 0.f;
     bool ok = true;
     for (int j = 0; j < nblk; ++j) {
-      const int sb = j & 1;
-      ok = wait_warp(&bar[B_SFULL + sb], (j >> 1) & 1, abort_flag, status);
+      ok = wait_warp(&bar[B_SFULL + t], j & 1, abort_flag, status);
       if (!ok) break;
       tc_fence_after();
       float s[BN];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(lane_base + sb * 128 + c * 32, s + c * 32);
+      for (int c = 0; c < 4; ++c) tmem_ld32(s_col + c * 32, s + c * 32);
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld_wait32(s + c * 32);
       const int lim = kv_len - j * BN;  // valid keys in this block
@@ -335,10 +531,7 @@ __global__ void __launch_bounds__(kRope ? 256 : 192, 1)
         for (int c = 0; c < BN; ++c)
           if (c >= lim) s[c] = -INFINITY;
       }
-      float mx = s[0];
-#pragma unroll
-      for (int c = 1; c < BN; ++c) mx = fmaxf(mx, s[c]);
-      mx *= c2;
+      const float mx = rowmax128(s) * c2;
       bool need = false;
       if (j == 0) {
         m_run = mx;
@@ -346,59 +539,50 @@ __global__ void __launch_bounds__(kRope ? 256 : 192, 1)
         need = mx > m_run + RESCALE_LOG2;
       }
       if (__any_sync(0xffffffffu, need)) {
+        // S_t(j) complete implies PV_t(j-1) complete (issued before it), so
+        // O holds exactly blocks 0..j-1 here.
         const float m_new = need ? mx : m_run;
         const float alpha = ex2(m_run - m_new);
-        // O holds blocks 0..j-1 only after PV(j-1) has completed.
-        ok = wait_warp(&bar[B_ODONE], (j - 1) & 1, abort_flag, status);
-        if (!ok) break;
-        tc_fence_after();
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           float o[32];
-          tmem_ld32(lane_base + TM_O + c * 32, o);
+          tmem_ld32(o_col + c * 32, o);
           tmem_ld_wait32(o);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] *= alpha;
-          tmem_st32(lane_base + TM_O + c * 32, o);
+          for (int e = 0; e < 32; e += 2) {
+            const float2 v =
+                ffma2(make_float2(o[e], o[e + 1]),
+                      make_float2(alpha, alpha), make_float2(0.f, 0.f));
+            o[e] = v.x;
+            o[e + 1] = v.y;
+          }
+          tmem_st32(o_col + c * 32, o);
         }
-        tmem_st_wait();
         l_run *= alpha;
         m_run = m_new;
       }
-      float sum = 0.f;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float p0 = ex2(fmaf(s[c * 32 + 2 * e], c2, -m_run));
-          const float p1 = ex2(fmaf(s[c * 32 + 2 * e + 1], c2, -m_run));
-          sum += p0 + p1;
-          pk[e] = pack_bf16x2(p0, p1);
-        }
-        // P (bf16 pairs) over the first 64 columns of this score buffer.
-        tmem_st16(lane_base + sb * 128 + c * 16, pk);
-      }
+      // P (bf16 pairs) over the first 64 columns of this tile's S buffer.
+      const float sum = (lim < BN)
+                            ? exp_store_row<false>(s, c2, m_run, s_col)
+                            : exp_store_row<true>(s, c2, m_run, s_col);
       l_run += sum;
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bar[B_PFULL + sb]);
+      if (lane == 0) mbar_arrive(&bar[B_PFULL + t]);
     }
-    // ODONE may be two phases behind here (only PV(nblk-3) is implied by
-    // the last score tile), so the final PV has a barrier of its own.
-    if (ok) ok = wait_warp(&bar[B_OFINAL], 0, abort_flag, status);
+    if (ok) ok = wait_warp(&bar[B_OFINAL + t], 0, abort_flag, status);
     if (ok) {
       tc_fence_after();
       const float inv = 1.0f / l_run;
-      const int row = q0 + r;
+      const int row = q0 + t * BM + r;
       __nv_bfloat16* orow =
           args.o + ((static_cast<int64_t>(b) * args.Lq + row) * args.heads +
                     head) * HD;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         float o[32];
-        tmem_ld32(lane_base + TM_O + c * 32, o);
+        tmem_ld32(o_col + c * 32, o);
         tmem_ld_wait32(o);
         uint32_t pk[16];
 #pragma unroll
@@ -413,30 +597,11 @@ __global__ void __launch_bounds__(kRope ? 256 : 192, 1)
         }
       }
     }
-  } else if (kRope) {
-    // -------------------------------------------------------------- RoPE --
-    const int t = threadIdx.x - 192;  // rows t and t + 64 of each tile
-    bool ok = wait_warp(&bar[B_QFULL], 0, abort_flag, status);
-    if (ok) {
-      for (int r = t; r < BM; r += kRopeThreads)
-        if (q0 + r < args.Lq) rope_row(sQ, r, q0 + r, args);
-      fence_proxy_async_smem();
-      mbar_arrive(&bar[B_QREADY]);
-    }
-    for (int j = 0; j < nblk && ok; ++j) {
-      const int st = j % NS;
-      ok = wait_warp(&bar[B_KFULL + st], (j / NS) & 1, abort_flag, status);
-      if (!ok) break;
-      for (int r = t; r < BN; r += kRopeThreads)
-        if (j * BN + r < kv_len) rope_row(sK + st * TILE, r, j * BN + r, args);
-      fence_proxy_async_smem();
-      mbar_arrive(&bar[B_KREADY + st]);
-    }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
   }
@@ -493,23 +658,35 @@ template <int kRope>
 int launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
            const AttnArgs& a, int B, cudaStream_t s) {
   static std::mutex mu;
-  static bool attr_set[64];
+  static int state[64];  // 0 unknown, 1 ready, 2 unusable
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
     return WAN_ECUDA;
   {
     std::lock_guard<std::mutex> lock(mu);
-    if (!attr_set[dev]) {
-      if (cudaFuncSetAttribute(attn_fwd_kernel<kRope>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               SMEM_DYN) != cudaSuccess)
+    if (state[dev] == 0) {
+      // setmaxnreg draws on the registers the CTA was launched with: refuse
+      // to launch if the compiled register count cannot fund the split
+      // (the .inc would otherwise wait forever).
+      cudaFuncAttributes fa;
+      if (cudaFuncGetAttributes(&fa, attn_fwd_kernel<kRope>) != cudaSuccess)
         return WAN_ECUDA;
-      attr_set[dev] = true;
+      const int need = 8 * 32 * kSoftmaxRegs + 4 * 32 * kOtherRegs;
+      if (fa.numRegs * kThreads < need) {
+        state[dev] = 2;
+      } else if (cudaFuncSetAttribute(
+                     attn_fwd_kernel<kRope>,
+                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                     SMEM_DYN) != cudaSuccess) {
+        return WAN_ECUDA;
+      } else {
+        state[dev] = 1;
+      }
     }
+    if (state[dev] != 1) return WAN_EUNSUPPORTED;
   }
-  dim3 grid((a.Lq + BM - 1) / BM, a.heads, B);
-  attn_fwd_kernel<kRope><<<grid, kRope ? 256 : 192, SMEM_DYN, s>>>(mq, mk, mv,
-                                                                   a);
+  dim3 grid((a.Lq + QT * BM - 1) / (QT * BM), a.heads, B);
+  attn_fwd_kernel<kRope><<<grid, kThreads, SMEM_DYN, s>>>(mq, mk, mv, a);
   return cudaGetLastError() == cudaSuccess ? WAN_OK : WAN_ECUDA;
 }
 
