@@ -104,6 +104,21 @@ def test_self_attn_identical_keys_mean_v():
     assert_attn_close(got, want, "identical keys")
 
 
+@pytest.mark.parametrize("L", [256, 200, 300])
+def test_self_attn_constant_negative_scores_exact(L):
+    # Every score equal and negative, every V row equal: softmax weights are
+    # uniform, O must be that V row bit for bit.  P = 2^(s - max) is then
+    # exactly 1 in every lane, so any error in the running row max (it must
+    # equal the negative score, not 0) shows up as a bf16 rounding change.
+    B, H = 1, 2
+    k0 = inputs.randn_bf16((1, 1, H, 128), 31)
+    k = k0.expand(B, L, H, 128).contiguous()
+    q = (-k0).expand(B, L, H, 128).contiguous()
+    v = inputs.randn_bf16((1, 1, H, 128), 32).expand(B, L, H, 128).contiguous()
+    got = _run_self(q, k, v, (1, 1, L), "none")
+    assert np.array_equal(got, f64(v))
+
+
 def test_self_attn_peaked_softmax():
     # Q x 8: scores spread ~8, softmax far from flat -- a kernel that returned
     # mean(V) or mixed rows up fails here.  Unrotated path: the rotated q, k

@@ -212,16 +212,31 @@ __device__ __forceinline__ void rope_row(uint8_t* tile, int r, int n,
   }
 }
 
-// Row max of 128 scores with 3-input max and four independent chains.
+// Row max of 128 scores with plain 2-input max and eight independent
+// chains: used for blocks whose masked entries hold -inf.
+__device__ __forceinline__ float rowmax128_masked(const float* s) {
+  float m[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) m[i] = s[i];
+#pragma unroll
+  for (int c = 8; c < BN; ++c) m[c & 7] = fmaxf(m[c & 7], s[c]);
+  return fmaxf(fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3])),
+               fmaxf(fmaxf(m[4], m[5]), fmaxf(m[6], m[7])));
+}
+
+// Row max of 128 finite scores with 3-input max and four independent chains:
+// s[0..3] seed the chains, s[4..123] go 8 per step, s[124..127] close them.
 __device__ __forceinline__ float rowmax128(const float* s) {
   float m0 = s[0], m1 = s[1], m2 = s[2], m3 = s[3];
 #pragma unroll
-  for (int c = 4; c < BN; c += 8) {
+  for (int c = 4; c + 8 <= BN - 4; c += 8) {
     m0 = fmax3(m0, s[c + 0], s[c + 1]);
     m1 = fmax3(m1, s[c + 2], s[c + 3]);
     m2 = fmax3(m2, s[c + 4], s[c + 5]);
     m3 = fmax3(m3, s[c + 6], s[c + 7]);
   }
+  m0 = fmax3(m0, s[BN - 4], s[BN - 3]);
+  m1 = fmax3(m1, s[BN - 2], s[BN - 1]);
   return fmaxf(fmax3(m0, m1, m2), m3);
 }
 
@@ -526,12 +541,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld_wait32(s + c * 32);
       const int lim = kv_len - j * BN;  // valid keys in this block
+      float mx;
       if (lim < BN) {
 #pragma unroll
         for (int c = 0; c < BN; ++c)
           if (c >= lim) s[c] = -INFINITY;
+        mx = rowmax128_masked(s);
+      } else {
+        mx = rowmax128(s);
       }
-      const float mx = rowmax128(s) * c2;
+      mx *= c2;
       bool need = false;
       if (j == 0) {
         m_run = mx;
