@@ -55,8 +55,8 @@ constexpr uint32_t SMEM_DYN = TILE * (QT + NSK + NSV) + 1024;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TM_O = 256;               // O of tile t at TM_O + 128 t
 constexpr int kThreads = 384;
-constexpr int kSoftmaxRegs = 216;            // warps 0-7
-constexpr int kOtherRegs = 72;               // warps 8-11
+constexpr int kSoftmaxRegs = 208;            // warps 0-7
+constexpr int kOtherRegs = 88;               // warps 8-11
 constexpr int kRopeThreads = 64;             // warps 10-11
 constexpr int MAX_CROSS_BATCH = 512;
 constexpr float RESCALE_LOG2 = 8.0f;         // rescale O when max grows > 2^8
@@ -212,31 +212,35 @@ __device__ __forceinline__ void rope_row(uint8_t* tile, int r, int n,
   }
 }
 
-// Row max of 128 scores with plain 2-input max and eight independent
-// chains: used for blocks whose masked entries hold -inf.
-__device__ __forceinline__ float rowmax128_masked(const float* s) {
+// Max of N scores with plain 2-input max and eight independent chains:
+// used for blocks whose masked entries hold -inf.
+template <int N>
+__device__ __forceinline__ float rowmax_masked(const float* s) {
+  static_assert(N % 8 == 0 && N >= 8, "N");
   float m[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) m[i] = s[i];
 #pragma unroll
-  for (int c = 8; c < BN; ++c) m[c & 7] = fmaxf(m[c & 7], s[c]);
+  for (int c = 8; c < N; ++c) m[c & 7] = fmaxf(m[c & 7], s[c]);
   return fmaxf(fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3])),
                fmaxf(fmaxf(m[4], m[5]), fmaxf(m[6], m[7])));
 }
 
-// Row max of 128 finite scores with 3-input max and four independent chains:
-// s[0..3] seed the chains, s[4..123] go 8 per step, s[124..127] close them.
-__device__ __forceinline__ float rowmax128(const float* s) {
+// Max of N finite scores with 3-input max and four independent chains:
+// s[0..3] seed the chains, s[4..N-5] go 8 per step, s[N-4..N-1] close them.
+template <int N>
+__device__ __forceinline__ float rowmax(const float* s) {
+  static_assert(N % 8 == 0 && N >= 16, "N");
   float m0 = s[0], m1 = s[1], m2 = s[2], m3 = s[3];
 #pragma unroll
-  for (int c = 4; c + 8 <= BN - 4; c += 8) {
+  for (int c = 4; c + 8 <= N - 4; c += 8) {
     m0 = fmax3(m0, s[c + 0], s[c + 1]);
     m1 = fmax3(m1, s[c + 2], s[c + 3]);
     m2 = fmax3(m2, s[c + 4], s[c + 5]);
     m3 = fmax3(m3, s[c + 6], s[c + 7]);
   }
-  m0 = fmax3(m0, s[BN - 4], s[BN - 3]);
-  m1 = fmax3(m1, s[BN - 2], s[BN - 1]);
+  m0 = fmax3(m0, s[N - 4], s[N - 3]);
+  m1 = fmax3(m1, s[N - 2], s[N - 1]);
   return fmaxf(fmax3(m0, m1, m2), m3);
 }
 
@@ -335,7 +339,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     setmaxnreg_dec();
     if (warp == 8) {
       // ------------------------------------------------------ TMA producer --
-      if (lane == 0) {
+      const bool leader = elect_one();
+      if (leader) {
         prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_k);
         prefetch_tmap(&tm_v);
@@ -354,7 +359,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (uk > 0)
           ok = wait_warp(&bar[B_KEMPTY + sk], (uk - 1) & 1, abort_flag, status);
         if (!ok) break;
-        if (lane == 0) {
+        if (leader) {
           mbar_expect_tx(&bar[B_KFULL + sk], TILE);
           tma_load_4d(sK + sk * TILE, &tm_k, &bar[B_KFULL + sk], 0, head,
                       j * BN, b);
@@ -366,7 +371,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (uv > 0)
           ok = wait_warp(&bar[B_VEMPTY + sv], (uv - 1) & 1, abort_flag, status);
         if (!ok) break;
-        if (lane == 0) {
+        if (leader) {
           mbar_expect_tx(&bar[B_VFULL + sv], TILE);
           tma_load_4d(sV + sv * TILE, &tm_v, &bar[B_VFULL + sv], 0, head,
                       j * BN, b);
@@ -386,42 +391,61 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     } else if (warp == 9) {
       // -------------------------------------------------------- MMA issuer --
-      const uint32_t sQa = smem_u32(sQ);
-      const uint32_t sKa = smem_u32(sK);
-      const uint32_t sVa = smem_u32(sV);
-      // S_t(j) = Q_t K(j)^T into the score buffer of tile t.
+      // Base descriptors, built once.  Per K step only a compile-time offset
+      // (bytes >> 4) is added to the start-address field, which cannot carry
+      // out of its 14 bits because shared addresses stay below 256 KB; this
+      // keeps the single issuing thread far ahead of the tensor core.
+      const uint64_t dq = sdesc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t dk = sdesc_sw128(smem_u32(sK), 16, 1024);
+      const uint64_t dv = sdesc_sw128(smem_u32(sV), HALF, 1024);
+      const bool leader = elect_one();
+      // S_t(j) = Q_t K(j)^T into the score buffer of tile t.  Descriptor
+      // arithmetic runs in all lanes (warp-uniform); one lane issues.
       auto issue_s = [&](int t, int j) {
-        const int sk = j % NSK;
-  #pragma unroll
-        for (int k = 0; k < HD / 16; ++k) {
-          // K-major operands: 16-channel K slices are 32 B apart inside a
-          // 128-B swizzle row; the second 64-channel half starts 16 KB on.
-          const uint32_t off = (k >> 2) * HALF + (k & 3) * 32;
-          const uint64_t adesc = sdesc_sw128(sQa + t * TILE + off, 16, 1024);
-          const uint64_t bdesc = sdesc_sw128(sKa + sk * TILE + off, 16, 1024);
-          umma_ss(tmem + t * 128, adesc, bdesc, IDESC_S, k > 0 ? 1u : 0u);
+        const uint64_t a0 = dq + ((t * TILE) >> 4);
+        const uint64_t b0 = dk + (((j % NSK) * TILE) >> 4);
+        const uint32_t d = tmem + t * 128;
+        if (leader) {
+#pragma unroll
+          for (int k = 0; k < HD / 16; ++k) {
+            // K-major operands: 16-channel K slices are 32 B apart inside a
+            // 128-B swizzle row; the second 64-channel half starts 16 KB on.
+            const uint32_t off = ((k >> 2) * HALF + (k & 3) * 32) >> 4;
+            umma_ss(d, a0 + off, b0 + off, IDESC_S, k > 0 ? 1u : 0u);
+          }
+          umma_commit(&bar[B_SFULL + t]);
         }
-        umma_commit(&bar[B_SFULL + t]);
+        __syncwarp();
       };
       // O_t += P_t(i) V(i).
       auto issue_pv = [&](int t, int i) {
-        const int sv = i % NSV;
-  #pragma unroll
-        for (int k = 0; k < BN / 16; ++k) {
+        const uint64_t b0 = dv + (((i % NSV) * TILE) >> 4);
+        const uint32_t d = tmem + TM_O + t * 128;
+        const uint32_t a = tmem + t * 128;
+        const uint32_t acc = i > 0 ? 1u : 0u;
+        if (leader) {
           // B = V[16k .. 16k+15][0..127]: MN-major, 8-key groups 1024 B
           // apart (SBO), the two 64-channel halves 16 KB apart (LBO).
-          const uint64_t bdesc =
-              sdesc_sw128(sVa + sv * TILE + k * 2048, HALF, 1024);
-          umma_ts(tmem + TM_O + t * 128, tmem + t * 128 + k * 8, bdesc,
-                  IDESC_PV, (i > 0 || k > 0) ? 1u : 0u);
+          umma_ts(d, a, b0, IDESC_PV, acc);
+#pragma unroll
+          for (int k = 1; k < BN / 16; ++k)
+            umma_ts(d, a + k * 8, b0 + ((k * 2048) >> 4), IDESC_PV, 1u);
         }
+        __syncwarp();
+      };
+      // Arrive on `b` when all MMAs issued so far are done (one lane).
+      auto commit = [&](uint64_t* b) {
+        if (leader) umma_commit(b);
+        __syncwarp();
       };
       // Waits for P_0(i) and V(i), clears text-padding rows of V(i).
+      // V(i) is waited for first: it does not depend on the softmax, so the
+      // issue of PV_0(i) follows P_0(i) as closely as possible.
       auto ready_pv0 = [&](int i) -> bool {
-        if (!wait_warp(&bar[B_PFULL + 0], i & 1, abort_flag, status))
-          return false;
         if (!wait_warp(&bar[B_VFULL + i % NSV], (i / NSV) & 1, abort_flag,
                        status))
+          return false;
+        if (!wait_warp(&bar[B_PFULL + 0], i & 1, abort_flag, status))
           return false;
         if (args.cross && kv_len < (i + 1) * BN) {
           // Text padding rows may hold anything (NaN included): P is 0 there
@@ -447,53 +471,40 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (j > 0) {
           ok = ready_pv0(j - 1);
           if (!ok) break;
-          if (lane == 0) issue_pv(0, j - 1);
-          __syncwarp();
+          issue_pv(0, j - 1);
         }
         ok = wait_warp(&bar[(kRope ? B_KREADY : B_KFULL) + sk], (j / NSK) & 1,
                        abort_flag, status);
         if (!ok) break;
         tc_fence_after();
-        if (lane == 0) issue_s(0, j);
-        __syncwarp();
+        issue_s(0, j);
         if (j > 0) {
           ok = wait_warp(&bar[B_PFULL + 1], (j - 1) & 1, abort_flag, status);
           if (!ok) break;
           tc_fence_after();
-          if (lane == 0) {
-            issue_pv(1, j - 1);
-            umma_commit(&bar[B_VEMPTY + (j - 1) % NSV]);
-          }
-          __syncwarp();
+          issue_pv(1, j - 1);
+          commit(&bar[B_VEMPTY + (j - 1) % NSV]);
         }
-        if (lane == 0) {
-          issue_s(1, j);
-          umma_commit(&bar[B_KEMPTY + sk]);
-        }
-        __syncwarp();
+        issue_s(1, j);
+        commit(&bar[B_KEMPTY + sk]);
       }
       if (ok) {
         const int i = nblk - 1;
         ok = ready_pv0(i);
-        if (ok && lane == 0) {
+        if (ok) {
           issue_pv(0, i);
-          umma_commit(&bar[B_OFINAL + 0]);
+          commit(&bar[B_OFINAL + 0]);
+          ok = wait_warp(&bar[B_PFULL + 1], i & 1, abort_flag, status);
         }
-        __syncwarp();
-        if (ok) ok = wait_warp(&bar[B_PFULL + 1], i & 1, abort_flag, status);
         if (ok) {
           tc_fence_after();
-          if (lane == 0) {
-            issue_pv(1, i);
-            umma_commit(&bar[B_OFINAL + 1]);
-            umma_commit(&bar[B_VEMPTY + i % NSV]);
-          }
+          issue_pv(1, i);
+          commit(&bar[B_OFINAL + 1]);
+          commit(&bar[B_VEMPTY + i % NSV]);
         }
-        __syncwarp();
       }
       // Drain every MMA before tensor memory is released.
-      if (lane == 0) umma_commit(&bar[B_DRAIN]);
-      __syncwarp();
+      commit(&bar[B_DRAIN]);
       wait_warp_drain(&bar[B_DRAIN], 0, status);
     } else if (kRope) {
       // -------------------------------------------------------------- RoPE --
@@ -541,49 +552,53 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld_wait32(s + c * 32);
       const int lim = kv_len - j * BN;  // valid keys in this block
-      float mx;
-      if (lim < BN) {
+      const bool masked = lim < BN;
+      if (masked) {
 #pragma unroll
         for (int c = 0; c < BN; ++c)
           if (c >= lim) s[c] = -INFINITY;
-        mx = rowmax128_masked(s);
-      } else {
-        mx = rowmax128(s);
       }
-      mx *= c2;
-      bool need = false;
+      float sum;
       if (j == 0) {
-        m_run = mx;
+        m_run = (masked ? rowmax_masked<BN>(s) : rowmax<BN>(s)) * c2;
+        sum = masked ? exp_store_row<false>(s, c2, m_run, s_col)
+                     : exp_store_row<true>(s, c2, m_run, s_col);
       } else {
-        need = mx > m_run + RESCALE_LOG2;
-      }
-      if (__any_sync(0xffffffffu, need)) {
-        // S_t(j) complete implies PV_t(j-1) complete (issued before it), so
-        // O holds exactly blocks 0..j-1 here.
-        const float m_new = need ? mx : m_run;
-        const float alpha = ex2(m_run - m_new);
+        // Exponentiate against the running max right away and find this
+        // block's max alongside: with no rescale the exponents stay <= 8
+        // (p <= 256, exact after the final O / l).  Only when some row's max
+        // grew by more than 2^8 is O rescaled and P formed again.
+        const float mx = (masked ? rowmax_masked<BN>(s) : rowmax<BN>(s)) * c2;
+        sum = masked ? exp_store_row<false>(s, c2, m_run, s_col)
+                     : exp_store_row<true>(s, c2, m_run, s_col);
+        const bool need = mx > m_run + RESCALE_LOG2;
+        if (__any_sync(0xffffffffu, need)) {
+          // S_t(j) complete implies PV_t(j-1) complete (issued before it),
+          // so O holds exactly blocks 0..j-1 here.
+          const float m_new = need ? mx : m_run;
+          const float alpha = ex2(m_run - m_new);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          float o[32];
-          tmem_ld32(o_col + c * 32, o);
-          tmem_ld_wait32(o);
+          for (int c = 0; c < 4; ++c) {
+            float o[32];
+            tmem_ld32(o_col + c * 32, o);
+            tmem_ld_wait32(o);
 #pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const float2 v =
-                ffma2(make_float2(o[e], o[e + 1]),
-                      make_float2(alpha, alpha), make_float2(0.f, 0.f));
-            o[e] = v.x;
-            o[e + 1] = v.y;
+            for (int e = 0; e < 32; e += 2) {
+              const float2 v =
+                  ffma2(make_float2(o[e], o[e + 1]),
+                        make_float2(alpha, alpha), make_float2(0.f, 0.f));
+              o[e] = v.x;
+              o[e + 1] = v.y;
+            }
+            tmem_st32(o_col + c * 32, o);
           }
-          tmem_st32(o_col + c * 32, o);
+          l_run *= alpha;
+          m_run = m_new;
+          tmem_st_wait();  // the first P stores land before they are redone
+          sum = masked ? exp_store_row<false>(s, c2, m_run, s_col)
+                       : exp_store_row<true>(s, c2, m_run, s_col);
         }
-        l_run *= alpha;
-        m_run = m_new;
       }
-      // P (bf16 pairs) over the first 64 columns of this tile's S buffer.
-      const float sum = (lim < BN)
-                            ? exp_store_row<false>(s, c2, m_run, s_col)
-                            : exp_store_row<true>(s, c2, m_run, s_col);
       l_run += sum;
       tmem_st_wait();
       tc_fence_before();

@@ -81,9 +81,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // Warp-uniform bounded wait for the completion of phase `parity` of `bar`.
 // Every lane of the warp must call it.  Once a phase has completed it stays
 // visible to the waiter until the waiter itself helps complete the next one,
-// so one lane seeing it is enough for the whole warp.  Gives up (returns
-// false) when the CTA-wide abort flag is set or after kWaitLimitNs, in which
-// case it sets the abort flag and stores WAN_ETIMEOUT in *status.
+// so as soon as one lane sees it, the lanes that have not yet seen it poll
+// once more and succeed (each successful try_wait is an acquire for that
+// lane).  Gives up (returns false) when the CTA-wide abort flag is set or
+// after kWaitLimitNs, in which case it sets the abort flag and stores
+// WAN_ETIMEOUT in *status.
 __device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity,
                                           volatile int* abort_flag,
                                           int* status) {
@@ -91,8 +93,11 @@ __device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity,
   const int lane = threadIdx.x & 31;
   uint64_t t0 = 0;
   for (uint32_t it = 0;; ++it) {
-    const bool ok = mbar_try_wait(a, parity);
-    if (__any_sync(0xffffffffu, ok)) return true;
+    bool done = mbar_try_wait(a, parity);
+    if (__any_sync(0xffffffffu, done)) {
+      if (!done) done = mbar_try_wait(a, parity);
+      if (__all_sync(0xffffffffu, done)) return true;
+    }
     if ((it & 31u) == 31u) {
       int bad = 0;
       if (lane == 0) {
@@ -123,8 +128,11 @@ __device__ __forceinline__ bool wait_warp_drain(uint64_t* bar,
   const int lane = threadIdx.x & 31;
   uint64_t t0 = 0;
   for (uint32_t it = 0;; ++it) {
-    const bool ok = mbar_try_wait(a, parity);
-    if (__any_sync(0xffffffffu, ok)) return true;
+    bool done = mbar_try_wait(a, parity);
+    if (__any_sync(0xffffffffu, done)) {
+      if (!done) done = mbar_try_wait(a, parity);
+      if (__all_sync(0xffffffffu, done)) return true;
+    }
     if ((it & 31u) == 31u) {
       int bad = 0;
       if (lane == 0) {
@@ -139,6 +147,19 @@ __device__ __forceinline__ bool wait_warp_drain(uint64_t* bar,
       if (__shfl_sync(0xffffffffu, bad, 0)) return false;
     }
   }
+}
+
+// One lane of the (converged) warp: true in exactly one lane.  Used instead
+// of a lane-index test so that the code around the elected instruction stays
+// warp-uniform (tcgen05.mma issue slows several-fold when the issuing code
+// runs divergent under a lane test while other warps share the scheduler).
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
 }
 
 // --- fences ---
