@@ -33,9 +33,6 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-HOST_GBS_FALLBACK = None
-
-
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
@@ -46,6 +43,10 @@ def parse():
     p.add_argument("--impl", choices=["wan", "reference"], default="wan")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-hbm", action="store_true",
+                   help="skip the HBM-bound kernel rooflines")
+    p.add_argument("--hbm-elems", type=int, default=1 << 28,
+                   help="fp32 elements per buffer of the fm_step roofline")
     p.add_argument("--cpu-rows", type=int, default=4096,
                    help="query rows of one head timed on the oracle")
     return p.parse_args()
@@ -191,6 +192,78 @@ def run_reference(args, w, rank, world):
 
 
 # ------------------------------------------------------------------- wan ---
+
+def hbm_rooflines(dev, g, L, H, n_lat, peak_gbs, n=1 << 28, reps=20):
+    """Achieved bandwidth of the two HBM-bound kernels, timed alone with CUDA
+    events: the fused CFG + Euler step on n-element fp32 buffers (default
+    2^28: 4 GiB of traffic per call, far above L2) and the RoPE pass on the
+    workload's Q and K; plus the step on the workload's own latent, timed
+    cold (L2 flushed by a 512 MiB write before every call)."""
+    import torch
+
+    from video_diffusion_transformer_self_b200 import wan
+
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(4242)
+    out = {}
+    x = torch.randn(n, device=dev, generator=gen)
+    c = torch.randn(n, device=dev, generator=gen)
+    u = torch.randn(n, device=dev, generator=gen)
+    for _ in range(3):
+        wan.fm_step(x, c, u, 4.0, 0.5, 0.49)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(reps):
+        wan.fm_step(x, c, u, 4.0, 0.5, 0.49)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    gbs = 16.0 * n / (ms / 1e3) / 1e9
+    out["fm_step_cfg"] = {"elements": n, "bytes_per_call": 16 * n,
+                          "ms": ms, "achieved_gbs": gbs, "peak_gbs": peak_gbs,
+                          "frac": gbs / peak_gbs}
+    del x, c, u
+    q = torch.randn(1, L, H, 128, device=dev, generator=gen).to(torch.bfloat16)
+    k = torch.randn(1, L, H, 128, device=dev, generator=gen).to(torch.bfloat16)
+    table = wan.rope3d_table(g)
+    for _ in range(3):
+        wan.rope3d_qk(q, k, g, table)
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(reps):
+        wan.rope3d_qk(q, k, g, table)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    nbytes = 4 * q.numel() * 2
+    gbs = nbytes / (ms / 1e3) / 1e9
+    out["rope3d_qk"] = {"tokens": L, "heads": H, "bytes_per_call": nbytes,
+                        "ms": ms, "achieved_gbs": gbs, "peak_gbs": peak_gbs,
+                        "frac": gbs / peak_gbs}
+    del q, k
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    xl = torch.randn(n_lat, device=dev, generator=gen)
+    cl = torch.randn(n_lat, device=dev, generator=gen)
+    ul = torch.randn(n_lat, device=dev, generator=gen)
+    tot = 0.0
+    for i in range(reps + 3):
+        flush.fill_(i & 255)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        wan.fm_step(xl, cl, ul, 4.0, 0.5, 0.49)
+        b.record()
+        torch.cuda.synchronize()
+        if i >= 3:
+            tot += a.elapsed_time(b)
+    ms = tot / reps
+    out["fm_step_latent_cold"] = {"elements": n_lat, "ms": ms,
+                                  "achieved_gbs": 16.0 * n_lat / (ms / 1e3)
+                                  / 1e9, "l2": "flushed before each call"}
+    return out
+
 
 def run_wan(args, w, rank, world, local_rank):
     import numpy as np
@@ -375,6 +448,10 @@ def run_wan(args, w, rank, world, local_rank):
         "e2e": e2e,
         "clocks": clk,
     }
+    if not args.no_hbm and world == 1:
+        line["hbm_kernels"] = hbm_rooflines(
+            dev, g, L, H, n_lat, float(pk.get("hbm_gbs", 6650.0)),
+            n=args.hbm_elems)
     if not args.no_cpu_baseline and world == 1:
         dt, fl, text = cpu_oracle_sample(w, args.cpu_rows)
         line["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": "TFLOP/s",
