@@ -7,23 +7,27 @@
 // come from the table wan_rope3d_table() writes (rows of 22 pairs: time,
 // height with a trailing pad, width with a leading pad).
 //
-// HBM-bound: each 16-byte chunk (8 bf16 = 4 complex pairs) of Q / K is read
-// and written once; the table (<= 70 KB) stays in L1 / L2.  One thread per
-// chunk per trip, consecutive threads on consecutive chunks (coalesced),
-// grid-stride over both tensors.
+// HBM-bound: every 16-byte chunk (8 bf16 = 4 complex pairs) of Q / K is read
+// and written once.  One warp per token (grid-stride over B * L tokens): the
+// token's (f, h, w) is found once, lane l owns chunk c = l & 15 of every
+// head row, loads the 4 cos / sin pairs of that chunk once, and walks the
+// heads two at a time (lanes 0-15 head 2i, lanes 16-31 head 2i+1), so each
+// warp access covers 512 contiguous bytes.
 #include "wan_internal.cuh"
 
 namespace wan {
 namespace {
 
 constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kBatch = 4;  // head rows per lane per batch
 
 struct RopeArgs {
   uint4* q;
   uint4* k;
   const float4* table;  // rows of 11 float4 = 22 {cos, sin} pairs
-  int64_t chunks;       // chunks per tensor = B * L * heads * 16
-  int heads, F, H, W;
+  int64_t tokens;       // B * L
+  int L, heads, F, H, W;
 };
 
 __device__ __forceinline__ float2 bf16x2_to_float2(uint32_t v) {
@@ -33,62 +37,72 @@ __device__ __forceinline__ float2 bf16x2_to_float2(uint32_t v) {
   return r;
 }
 
-// Rotate the 4 complex pairs of one chunk.  `c` = chunk index in the head
-// row (0..15): absolute pairs p = 4c .. 4c+3.  tt / th / tw point at the
-// token's table rows (float4 = two pairs).
-__device__ __forceinline__ uint4 rotate_chunk(uint4 raw, int c,
-                                              const float4* tt,
-                                              const float4* th,
-                                              const float4* tw) {
-  uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    const int p0 = 4 * c + 2 * half;  // even absolute pair index
-    float4 cs;                        // {cos p0, sin p0, cos p0+1, sin p0+1}
-    if (p0 + 1 < 22) {
-      cs = tt[p0 >> 1];
-    } else if (p0 >= 22 && p0 + 1 < 43) {
-      cs = th[(p0 - 22) >> 1];
-    } else if (p0 >= 44) {
-      cs = tw[(p0 - 42) >> 1];
-    } else {  // p0 = 42: pair 42 is the last height pair, 43 the first width
-      const float4 a = th[10];  // entries 20, 21 -> pair 42 in .x/.y
-      const float4 b = tw[0];   // entries 0 (pad), 1 -> pair 43 in .z/.w
-      cs = make_float4(a.x, a.y, b.z, b.w);
-    }
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const float2 v = bf16x2_to_float2(w[2 * half + e]);
-      const float co = e ? cs.z : cs.x;
-      const float si = e ? cs.w : cs.y;
-      const float re = fmaf(v.x, co, -v.y * si);
-      const float im = fmaf(v.x, si, v.y * co);
-      w[2 * half + e] = pack_bf16x2(re, im);
-    }
-  }
-  return make_uint4(w[0], w[1], w[2], w[3]);
+// {cos, sin} of absolute pairs p0 and p0 + 1 (p0 even) for the token whose
+// band rows are tt (time), th (height), tw (width).
+__device__ __forceinline__ float4 pair_cs(int p0, const float4* tt,
+                                          const float4* th,
+                                          const float4* tw) {
+  if (p0 + 1 < 22) return __ldg(tt + (p0 >> 1));
+  if (p0 >= 22 && p0 + 1 < 43) return __ldg(th + ((p0 - 22) >> 1));
+  if (p0 >= 44) return __ldg(tw + ((p0 - 42) >> 1));
+  // p0 = 42: pair 42 is the last height pair, pair 43 the first width pair
+  const float4 lo = __ldg(th + 10);  // entries 20, 21 -> pair 42 in .x/.y
+  const float4 hi = __ldg(tw);       // entries 0 (pad), 1 -> pair 43 in .z/.w
+  return make_float4(lo.x, lo.y, hi.z, hi.w);
+}
+
+__device__ __forceinline__ uint32_t rot2(uint32_t v, float co, float si) {
+  const float2 x = bf16x2_to_float2(v);
+  return pack_bf16x2(fmaf(x.x, co, -x.y * si), fmaf(x.x, si, x.y * co));
+}
+
+__device__ __forceinline__ uint4 rotate_chunk(uint4 raw, float4 a, float4 b) {
+  return make_uint4(rot2(raw.x, a.x, a.y), rot2(raw.y, a.z, a.w),
+                    rot2(raw.z, b.x, b.y), rot2(raw.w, b.z, b.w));
 }
 
 __global__ void __launch_bounds__(kThreads) rope3d_kernel(RopeArgs a) {
-  const int64_t total = a.chunks * 2;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * kThreads;
+  const int lane = threadIdx.x & 31;
+  const int c = lane & 15;        // 16-byte chunk within a head row
+  const int hsub = lane >> 4;     // head parity handled by this half-warp
+  const int64_t wstride = static_cast<int64_t>(gridDim.x) * kWarps;
   const int hw = a.H * a.W;
-  for (int64_t g = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x;
-       g < total; g += stride) {
-    const bool is_k = g >= a.chunks;
-    const int64_t i = is_k ? g - a.chunks : g;
-    uint4* base = is_k ? a.k : a.q;
-    if (!base) continue;
-    const int c = static_cast<int>(i & 15);
-    const int64_t row = i >> 4;  // (b * L + n) * heads + head
-    const int n = static_cast<int>((row / a.heads) % (static_cast<int64_t>(a.F) * hw));
+  for (int64_t tok = static_cast<int64_t>(blockIdx.x) * kWarps +
+                     (threadIdx.x >> 5);
+       tok < a.tokens; tok += wstride) {
+    const int n = static_cast<int>(tok % a.L);
     const int f = n / hw;
     const int h = (n / a.W) % a.H;
     const int w = n % a.W;
     const float4* tt = a.table + static_cast<int64_t>(f) * 11;
     const float4* th = a.table + static_cast<int64_t>(a.F + h) * 11;
     const float4* tw = a.table + static_cast<int64_t>(a.F + a.H + w) * 11;
-    base[i] = rotate_chunk(base[i], c, tt, th, tw);
+    const float4 cs0 = pair_cs(4 * c, tt, th, tw);
+    const float4 cs1 = pair_cs(4 * c + 2, tt, th, tw);
+    const int64_t row0 = tok * a.heads;  // first head row of this token
+    // Batches of kBatch head rows per lane: all loads of a batch are issued
+    // before any rotation so that 2 * kBatch 16-byte loads are in flight.
+    for (int hh0 = hsub; hh0 < a.heads; hh0 += 2 * kBatch) {
+      uint4 vq[kBatch], vk[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int hh = hh0 + 2 * u;
+        const int64_t idx = (row0 + hh) * 16 + c;
+        if (hh < a.heads) {
+          if (a.q) vq[u] = a.q[idx];
+          if (a.k) vk[u] = a.k[idx];
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int hh = hh0 + 2 * u;
+        const int64_t idx = (row0 + hh) * 16 + c;
+        if (hh < a.heads) {
+          if (a.q) a.q[idx] = rotate_chunk(vq[u], cs0, cs1);
+          if (a.k) a.k[idx] = rotate_chunk(vk[u], cs0, cs1);
+        }
+      }
+    }
   }
 }
 
@@ -120,13 +134,13 @@ extern "C" int wan_rope3d_qk(void* q, void* k, int B, wan_grid_t g,
   a.q = static_cast<uint4*>(q);
   a.k = static_cast<uint4*>(k);
   a.table = static_cast<const float4*>(d_table);
-  const int64_t L = static_cast<int64_t>(g.F) * g.H * g.W;
-  a.chunks = static_cast<int64_t>(B) * L * heads * 16;
+  a.L = g.F * g.H * g.W;
+  a.tokens = static_cast<int64_t>(B) * a.L;
   a.heads = heads;
   a.F = g.F;
   a.H = g.H;
   a.W = g.W;
-  int64_t blocks = (2 * a.chunks + wan::kThreads - 1) / wan::kThreads;
+  int64_t blocks = (a.tokens + wan::kWarps - 1) / wan::kWarps;
   const int64_t cap = static_cast<int64_t>(sm_count[dev]) * 8;
   if (blocks > cap) blocks = cap;
   wan::rope3d_kernel<<<static_cast<unsigned>(blocks), wan::kThreads, 0,
