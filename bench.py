@@ -193,6 +193,35 @@ def run_reference(args, w, rank, world):
 
 # ------------------------------------------------------------------- wan ---
 
+# DRAM bytes per algorithmic byte (Q, K, V read once, O written once) of the
+# self-attention kernel, from the ncu capture of the 480p-81f launch:
+# 810.06 MB measured for 805.31 MB algorithmic.  The kernel's DRAM traffic
+# grows in proportion to B * L * heads, so a launch's traffic is this ratio
+# times its algorithmic bytes.
+ATTN_DRAM_PER_ALG_BYTE = 810.06 / 805.31
+
+
+def rank_seed_offset(rank):
+    """Seed offset of a rank's inputs: every rank runs its own problem."""
+    return 7919 * int(rank)
+
+
+def max_over_ranks(values, dist=None, device=None):
+    """Element-wise MAX of a list of floats over all ranks (identity at 1)."""
+    import torch
+    if dist is None:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64,
+                     device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def job_throughput(world, flops_per_step, steps, max_ms):
+    """Whole-job TFLOP/s: every rank's FLOPs over the slowest rank's time."""
+    return world * flops_per_step * steps / (max_ms / 1e3) / 1e12
+
+
 def hbm_rooflines(dev, g, L, H, n_lat, peak_gbs, n=1 << 28, reps=20):
     """Achieved bandwidth of the two HBM-bound kernels, timed alone with CUDA
     events: the fused CFG + Euler step on n-element fp32 buffers (default
@@ -280,7 +309,7 @@ def run_wan(args, w, rank, world, local_rank):
     B, H = w.batch, w.heads
     n_lat = int(np.prod(lat)) * B
     sigmas = wan.fm_sigmas(w.steps, w.shift)
-    seed_off = 7919 * rank  # every rank runs its own independent problem
+    seed_off = rank_seed_offset(rank)
 
     def sd(role):
         return inputs.seed_for(w.index, role) + seed_off
@@ -310,12 +339,13 @@ def run_wan(args, w, rank, world, local_rank):
 
     def step(i, timed):
         s0, s1 = sigmas[i % w.steps], sigmas[i % w.steps + 1]
+        if args.rope == "pre":
+            wan.rope3d_qk(d["q"], d["k"], g, table)
         if timed:
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
             e0.record(stream)
         if args.rope == "pre":
-            wan.rope3d_qk(d["q"], d["k"], g, table)
             wan.self_attn(d["q"], d["k"], d["v"], o, g)
         else:
             wan.self_attn(d["q"], d["k"], d["v"], o, g, table=table)
@@ -357,13 +387,10 @@ def run_wan(args, w, rank, world, local_rank):
     ms = t_start.elapsed_time(t_end)
     if wan.device_status() != 0:
         raise RuntimeError("device timeout during the timed steps")
-    # self-attention kernel time (includes the RoPE pass with --rope pre)
+    # self-attention launch time (the RoPE pass of --rope pre excluded)
     attn_ms = [a.elapsed_time(b) for a, b in ev_pairs]
     attn_avg = sum(attn_ms) / len(attn_ms)
-    if dist is not None:
-        t = torch.tensor([ms, attn_avg], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, attn_avg = float(t[0]), float(t[1])
+    ms, attn_avg = max_over_ranks([ms, attn_avg], dist, dev)
 
     # ----- end to end: host buffers in, results out, every step -----
     # Each step copies its inputs from pinned host memory and reads back its
@@ -439,13 +466,8 @@ def run_wan(args, w, rank, world, local_rank):
         e1 = run_steps(args.steps, start_ev=e0)
         torch.cuda.synchronize()
         barrier()
-        e2e_ms = e0.elapsed_time(e1)
-        if dist is not None:
-            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t[0])
-        e2e = {"value": world * flops_self * args.steps / (e2e_ms / 1e3)
-               / 1e12,
+        e2e_ms = max_over_ranks([e0.elapsed_time(e1)], dist, dev)[0]
+        e2e = {"value": job_throughput(world, flops_self, args.steps, e2e_ms),
                "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h,
                "ms_per_step": e2e_ms / args.steps,
@@ -455,7 +477,7 @@ def run_wan(args, w, rank, world, local_rank):
         return
     pk, pk_kind = peaks()
     peak = float(pk.get("bf16_tflops_sustained", 1400.0))
-    value = world * flops_self * args.steps / (ms / 1e3) / 1e12
+    value = job_throughput(world, flops_self, args.steps, ms)
     achieved = flops_self / (attn_avg / 1e3) / 1e12
     line = {
         "metric": "self-attn TFLOP/s",
@@ -484,10 +506,13 @@ def run_wan(args, w, rank, world, local_rank):
             "measured_sustained": value / peak,
         },
         "roofline": {
-            "kernel": "self_attn" + ("+rope3d_qk" if args.rope == "pre"
-                                     else " (fused RoPE)"),
+            "kernel": "attn_fwd_kernel self-attention" + (
+                "" if args.rope == "pre" else " with fused RoPE"),
             "bound": "tensor", "achieved": achieved, "peak": peak,
-            "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+            "unit": "TFLOP/s", "frac": achieved / peak,
+            "traffic": ATTN_DRAM_PER_ALG_BYTE * 4 * B * L * H * 256,
+            "traffic_source": "ncu dram read+write of the 480p-81f launch, "
+                              "scaled by bytes processed",
             "peak_kind": pk_kind + " sustained bf16 (kernel timed inside a "
                                    "long step)",
             "avg_launch_ms": attn_avg,
