@@ -75,3 +75,59 @@ def attention(q, k, v, scale, kv_lens=None, rows=None, row_block=512):
                 out[b, r0:r0 + row_block, h, :] = attend(qh, kh, vh, scale,
                                                          kv_len)
     return out
+
+
+# --------------------------------------------------------- block-causal --
+#
+# Long-video survey, section "Route 3 · Self Forcing": bidirectional full
+# attention is replaced by causal attention over chunks of frames so that a
+# finished chunk can be decoded and streamed; each new chunk attends to the
+# chunks before it through a KV cache (the KV cache can also be capped).
+#
+# Reading: a query at absolute token position a (frame-major order) belongs
+# to chunk floor(a / chunk_tokens) and sees every key j with
+#     j < (floor(a / chunk_tokens) + 1) * chunk_tokens,
+# i.e. all tokens of its own chunk and of every earlier chunk.  In the KV
+# cache form the queries of one chunk sit at absolute positions
+# q_offset .. q_offset + Lq - 1 and the keys are the cached prefix followed
+# by that chunk.
+
+def block_causal_limits(lq, lk, chunk_tokens, q_offset=0):
+    """Per-query key limit (exclusive) of the block-causal mask."""
+    if chunk_tokens < 1 or q_offset < 0 or q_offset + lq > lk:
+        raise ValueError("bad block-causal geometry")
+    a = q_offset + np.arange(lq)
+    return np.minimum(lk, (a // chunk_tokens + 1) * chunk_tokens)
+
+
+def attend_limited(q, k, v, scale, limits):
+    """One (batch, head) slice with a per-row key limit, fp64.
+
+    Row i uses keys 0 .. limits[i]-1 only (the definition above, evaluated
+    row by row).
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    out = np.empty((q.shape[0], v.shape[1]), dtype=np.float64)
+    for i, n in enumerate(limits):
+        s = (q[i] @ k[:n].T) * scale
+        p = np.exp(s - s.max())
+        out[i] = (p @ v[:n]) / p.sum()
+    return out
+
+
+def block_causal_attention(q, k, v, scale, chunk_tokens, q_offset=0,
+                           rows=None):
+    """Block-causal attention over [B, L, heads, d] tensors (fp64)."""
+    q = np.asarray(q)
+    b_, lq, nh, d = q.shape
+    lk = np.asarray(k).shape[1]
+    lim = block_causal_limits(lq, lk, chunk_tokens, q_offset)
+    rows = np.arange(lq) if rows is None else np.asarray(rows)
+    out = np.empty((b_, rows.shape[0], nh, d), dtype=np.float64)
+    for b in range(b_):
+        for h in range(nh):
+            out[b, :, h, :] = attend_limited(q[b, rows, h, :], k[b, :, h, :],
+                                             v[b, :, h, :], scale, lim[rows])
+    return out

@@ -151,3 +151,67 @@ def test_planted_transpose_mistake_is_caught(monkeypatch):
         return orig(q, k, k, scale, kv_len)
     monkeypatch.setattr(attention, "attend", wrong)
     assert np.max(np.abs(attention.attend(q, k, v, 0.5) - good)) > 1e-3
+
+
+# ------------------------------------------------------------ block-causal --
+
+def test_block_causal_one_chunk_is_full_attention():
+    r = _rng(21)
+    q, k, v = (r.standard_normal((1, 24, 2, 8)) for _ in range(3))
+    full = attention.attention(q, k, v, 0.4)
+    bc = attention.block_causal_attention(q, k, v, 0.4, chunk_tokens=24)
+    assert np.max(np.abs(bc - full)) < 1e-13
+    bc2 = attention.block_causal_attention(q, k, v, 0.4, chunk_tokens=1000)
+    assert np.max(np.abs(bc2 - full)) < 1e-13
+
+
+def test_block_causal_chunk_one_is_token_causal_sdpa():
+    # chunk of one token = ordinary causal attention (library routine)
+    r = _rng(22)
+    q, k, v = (r.standard_normal((2, 17, 3, 8)) for _ in range(3))
+    got = attention.block_causal_attention(q, k, v, 1 / math.sqrt(8), 1)
+    t = [torch.from_numpy(x).permute(0, 2, 1, 3) for x in (q, k, v)]
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        *t, is_causal=True).permute(0, 2, 1, 3).numpy()
+    assert np.max(np.abs(got - ref)) < 1e-12
+
+
+def test_block_causal_matches_explicit_mask_sdpa():
+    r = _rng(23)
+    L, chunk = 20, 6
+    q, k, v = (r.standard_normal((1, L, 2, 8)) for _ in range(3))
+    got = attention.block_causal_attention(q, k, v, 0.3, chunk)
+    mask = torch.zeros(L, L, dtype=torch.bool)
+    for a in range(L):
+        mask[a, :min(L, (a // chunk + 1) * chunk)] = True
+    t = [torch.from_numpy(x).permute(0, 2, 1, 3) for x in (q, k, v)]
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        *t, attn_mask=mask, scale=0.3).permute(0, 2, 1, 3).numpy()
+    assert np.max(np.abs(got - ref)) < 1e-12
+
+
+def test_block_causal_kv_cache_form_equals_full_rows():
+    # queries of the last chunk against cached keys = rows of the full run
+    r = _rng(24)
+    L, chunk = 30, 7
+    q, k, v = (r.standard_normal((1, L, 1, 8)) for _ in range(3))
+    full = attention.block_causal_attention(q, k, v, 0.5, chunk)
+    off = 21  # queries of positions 21..29 (chunks 3 and 4)
+    part = attention.block_causal_attention(q[:, off:], k, v, 0.5, chunk,
+                                            q_offset=off)
+    assert np.max(np.abs(part - full[:, off:])) < 1e-13
+    # the first chunk never sees later keys: changing them changes nothing
+    k2, v2 = k.copy(), v.copy()
+    k2[:, chunk:] += 5.0
+    v2[:, chunk:] -= 3.0
+    again = attention.block_causal_attention(q, k2, v2, 0.5, chunk)
+    assert np.array_equal(again[:, :chunk], full[:, :chunk])
+
+
+def test_block_causal_limits_and_rejects():
+    lim = attention.block_causal_limits(5, 9, 4, q_offset=4)
+    assert list(lim) == [8, 8, 8, 8, 9]
+    with pytest.raises(ValueError):
+        attention.block_causal_limits(5, 8, 4, q_offset=4)
+    with pytest.raises(ValueError):
+        attention.block_causal_limits(5, 9, 0)
