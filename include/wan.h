@@ -125,6 +125,26 @@ int wan_cross_attn(const void* q, const void* k_ctx, const void* v_ctx,
                    void* o, const int32_t* ctx_lens, int B, int Lq, int Lk,
                    int heads, int head_dim, float softmax_scale, void* s);
 
+/* ------------------------------------------------ block-causal (chunks) --
+ * Long-video survey (atlascloud.ai), section "Route 3 · Self Forcing":
+ * bidirectional attention is replaced by causal attention over chunks of
+ * frames, each chunk attending to earlier chunks through a KV cache.  A
+ * query at absolute token position a = q_offset + i sees keys
+ *   j < min(Lk, (floor(a / chunk_tokens) + 1) * chunk_tokens),
+ * i.e. its own chunk and all earlier ones:
+ *   O = softmax(Q K^T * softmax_scale + mask) V.
+ * Full sequence: q_offset = 0, Lq = Lk.  KV-cache step: the queries of one
+ * chunk (Lq tokens at absolute positions q_offset ..) against the cached
+ * keys followed by that chunk (Lk >= q_offset + Lq).  q, o: [B, Lq, heads,
+ * 128]; k, v: [B, Lk, heads, 128] bf16, already rotated (wan_rope3d_qk).
+ * chunk_tokens >= 1, q_offset >= 0, q_offset + Lq <= Lk.  Keys beyond a
+ * row's limit get weight exactly 0; as they can share a key block with
+ * visible keys they must be finite (0 * NaN would not vanish).             */
+int wan_block_causal_attn(const void* q, const void* k, const void* v,
+                          void* o, int B, int Lq, int Lk, int heads,
+                          int head_dim, int chunk_tokens, int q_offset,
+                          float softmax_scale, void* s);
+
 /* ------------------------------------------------------------- sampler --
  * Wan2.2 source reading, ch. 5, section "shift": the points are laid
  * uniformly and mapped by sigma = shift*s / (1 + (shift-1)*s); ch. 1

@@ -137,3 +137,12 @@ def test_argument_checks_without_device(lib):
         == wan.WAN_EINVAL
     assert L.wan_rope3d_qk(odd, None, 1, g, 2, 128, p, None) \
         == wan.WAN_EALIGN
+    o = ctypes.c_void_p(8192)
+    assert L.wan_block_causal_attn(p, p, p, o, 1, 10, 20, 2, 128, 0, 0, 0.1,
+                                   None) == wan.WAN_EINVAL  # chunk 0
+    assert L.wan_block_causal_attn(p, p, p, o, 1, 10, 20, 2, 128, 5, 11, 0.1,
+                                   None) == wan.WAN_EINVAL  # past the keys
+    assert L.wan_block_causal_attn(p, p, p, o, 1, 10, 20, 2, 128, 5, -1, 0.1,
+                                   None) == wan.WAN_EINVAL
+    assert L.wan_block_causal_attn(odd, p, p, o, 1, 10, 20, 2, 128, 5, 0, 0.1,
+                                   None) == wan.WAN_EALIGN

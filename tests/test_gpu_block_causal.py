@@ -1,0 +1,88 @@
+"""GPU parity of wan_block_causal_attn (chunk-wise causal attention with a
+KV cache) against the fp64 oracle."""
+
+import numpy as np
+import pytest
+import torch
+
+from gpu_common import (assert_attn_close, check_guards, cuda, f64,
+                        guarded_empty_like, scale_for)
+from oracle import attention as oattn
+from video_diffusion_transformer_self_b200 import build, inputs, wan
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    build.build()
+    wan.lib()
+
+
+def _run(q, k, v, chunk, q_offset=0):
+    qg, kg, vg = cuda(q), cuda(k), cuda(v)
+    o, buf, guard = guarded_empty_like(qg)
+    wan.block_causal_attn(qg, kg, vg, o, chunk, q_offset)
+    torch.cuda.synchronize()
+    assert wan.device_status() == 0
+    check_guards(buf, guard)
+    return f64(o)
+
+
+def _qkv(B, Lq, Lk, H, seed):
+    q = inputs.randn_bf16((B, Lq, H, 128), seed)
+    k = inputs.randn_bf16((B, Lk, H, 128), seed + 1)
+    v = inputs.randn_bf16((B, Lk, H, 128), seed + 2)
+    return q, k, v
+
+
+@pytest.mark.parametrize("B,L,H,chunk", [
+    (1, 300, 2, 50),     # chunks inside tiles, several per CTA
+    (2, 700, 1, 128),    # chunk = one key block
+    (1, 520, 2, 200),    # chunk boundaries mid-block
+    (1, 257, 1, 1),      # token-causal
+    (1, 333, 2, 333),    # one chunk = full attention
+    (1, 1000, 1, 2000),  # chunk longer than the sequence
+])
+def test_full_sequence(B, L, H, chunk):
+    q, k, v = _qkv(B, L, L, H, 500 + L)
+    got = _run(q, k, v, chunk)
+    want = oattn.block_causal_attention(f64(q), f64(k), f64(v), scale_for(),
+                                        chunk)
+    assert_attn_close(got, want, "block-causal L=%d chunk=%d" % (L, chunk))
+
+
+@pytest.mark.parametrize("chunk,n_chunks", [(120, 5), (1560, 3)])
+def test_kv_cache_chunk_step(chunk, n_chunks):
+    # the last chunk's queries against the cached prefix + itself
+    L = chunk * n_chunks
+    q, k, v = _qkv(1, L, L, 2, 900 + chunk)
+    off = L - chunk
+    got = _run(q[:, off:].contiguous(), k, v, chunk, q_offset=off)
+    want = oattn.block_causal_attention(f64(q[:, off:]), f64(k), f64(v),
+                                        scale_for(), chunk, q_offset=off)
+    assert_attn_close(got, want, "kv-cache chunk %d" % chunk)
+
+
+def test_first_chunk_ignores_later_keys():
+    chunk, L = 96, 400
+    q, k, v = _qkv(1, L, L, 1, 77)
+    k2 = (k.float() + 5.0).to(torch.bfloat16)
+    v2 = (v.float() - 3.0).to(torch.bfloat16)
+    k2[:, :chunk] = k[:, :chunk]
+    v2[:, :chunk] = v[:, :chunk]
+    a = _run(q[:, :chunk].contiguous(), k, v, chunk)
+    b = _run(q[:, :chunk].contiguous(), k2, v2, chunk)
+    # keys past the first chunk get weight exactly 0 (they may share a
+    # loaded key block with visible keys): changing them changes no bit
+    assert np.array_equal(a, b)
+
+
+def test_480p_17f_frame_chunks():
+    # 7,800 tokens, chunk = one latent frame (1,560 tokens), 12 heads
+    L, H, chunk = 7800, 12, 1560
+    q, k, v = _qkv(1, L, L, H, inputs.seed_for(1, "q"))
+    got = _run(q, k, v, chunk)
+    want = oattn.block_causal_attention(f64(q), f64(k), f64(v), scale_for(),
+                                        chunk)
+    assert_attn_close(got, want, "block-causal 7800")

@@ -73,6 +73,8 @@ struct AttnArgs {
   int F, H, W;          // token grid of the RoPE variant
   float scale_log2;     // softmax_scale * log2(e)
   int cross;            // 1: per-batch key length from lens[]
+  int chunk;            // > 0: block-causal, chunk length in tokens
+  int q_offset;         // block-causal: absolute position of query row 0
   int lens[MAX_CROSS_BATCH];
 };
 
@@ -292,10 +294,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int q0 = blockIdx.x * (QT * BM);
+  // Block-causal CTAs differ in work; the heaviest (last) start first.
+  const int tile_x = args.chunk ? (gridDim.x - 1 - blockIdx.x) : blockIdx.x;
+  const int q0 = tile_x * (QT * BM);
   const int head = blockIdx.y;
   const int b = blockIdx.z;
-  const int kv_len = args.cross ? args.lens[b] : args.Lk;
+  int kv_len = args.cross ? args.lens[b] : args.Lk;
+  if (args.chunk) {
+    // keys visible to the last query row of this CTA
+    const int last = min(q0 + QT * BM, args.Lq) - 1 + args.q_offset;
+    kv_len = min(args.Lk, (last / args.chunk + 1) * args.chunk);
+  }
   const int nblk = (kv_len + BN - 1) / BN;
   volatile int* abort_flag = &s_abort;
   int* status = &g_wan_status;
@@ -539,6 +548,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t s_col = lane_base + t * 128;
     const uint32_t o_col = lane_base + TM_O + t * 128;
     const float c2 = args.scale_log2;
+    // Keys this row may see: all kv_len, or its block-causal limit.
+    int row_lim = kv_len;
+    if (args.chunk && q0 + t * BM + r < args.Lq) {
+      const int a = q0 + t * BM + r + args.q_offset;
+      row_lim = min(args.Lk, (a / args.chunk + 1) * args.chunk);
+    }
     float m_run = -INFINITY;
     float l_run = 0.f;
     bool ok = true;
@@ -551,8 +566,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < 4; ++c) tmem_ld32(s_col + c * 32, s + c * 32);
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld_wait32(s + c * 32);
-      const int lim = kv_len - j * BN;  // valid keys in this block
-      const bool masked = lim < BN;
+      const int lim = row_lim - j * BN;  // valid keys of this row here
+      // warp-uniform: any masked row sends the warp down the exact path
+      const bool masked = __any_sync(0xffffffffu, lim < BN);
       if (masked) {
 #pragma unroll
         for (int c = 0; c < BN; ++c)
@@ -775,8 +791,41 @@ int wan_self_attn(const void* q, const void* k, const void* v, void* o,
   a.W = g.W;
   a.scale_log2 = softmax_scale * 1.4426950408889634f;
   a.cross = 0;
+  a.chunk = 0;
+  a.q_offset = 0;
   return d_table ? launch<1>(mq, mk, mv, a, B, as_stream(s))
                  : launch<0>(mq, mk, mv, a, B, as_stream(s));
+}
+
+int wan_block_causal_attn(const void* q, const void* k, const void* v,
+                          void* o, int B, int Lq, int Lk, int heads,
+                          int head_dim, int chunk_tokens, int q_offset,
+                          float softmax_scale, void* s) {
+  using namespace wan;
+  int st = check_common(q, k, v, o, B, Lq, Lk, heads, head_dim,
+                        softmax_scale);
+  if (st != WAN_OK) return st;
+  if (chunk_tokens < 1 || q_offset < 0 ||
+      static_cast<int64_t>(q_offset) + Lq > Lk)
+    return WAN_EINVAL;
+  st = check_device(nullptr);
+  if (st != WAN_OK) return st;
+  CUtensorMap mq, mk, mv;
+  if ((st = make_map(&mq, q, B, Lq, heads)) != WAN_OK) return st;
+  if ((st = make_map(&mk, k, B, Lk, heads)) != WAN_OK) return st;
+  if ((st = make_map(&mv, v, B, Lk, heads)) != WAN_OK) return st;
+  AttnArgs a;
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.table = nullptr;
+  a.Lq = Lq;
+  a.Lk = Lk;
+  a.heads = heads;
+  a.F = a.H = a.W = 1;
+  a.scale_log2 = softmax_scale * 1.4426950408889634f;
+  a.cross = 0;
+  a.chunk = chunk_tokens;
+  a.q_offset = q_offset;
+  return launch<0>(mq, mk, mv, a, B, as_stream(s));
 }
 
 int wan_cross_attn(const void* q, const void* k_ctx, const void* v_ctx,
@@ -804,6 +853,8 @@ int wan_cross_attn(const void* q, const void* k_ctx, const void* v_ctx,
   a.F = a.H = a.W = 1;
   a.scale_log2 = softmax_scale * 1.4426950408889634f;
   a.cross = 1;
+  a.chunk = 0;
+  a.q_offset = 0;
   for (int i = 0; i < B; ++i) a.lens[i] = ctx_lens[i];
   return launch<0>(mq, mk, mv, a, B, as_stream(s));
 }

@@ -55,6 +55,8 @@ _SIGNATURES = {
                            ctypes.c_float, _P]),
     "wan_cross_attn": (_I, [_P, _P, _P, _P, ctypes.POINTER(ctypes.c_int32),
                             _I, _I, _I, _I, _I, ctypes.c_float, _P]),
+    "wan_block_causal_attn": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I,
+                                   _I, ctypes.c_float, _P]),
     "wan_fm_sigmas": (_I, [_I, ctypes.c_double, ctypes.c_double,
                            ctypes.POINTER(ctypes.c_double)]),
     "wan_fm_step": (_I, [_P, _P, _P, ctypes.c_float, ctypes.c_int64,
@@ -185,6 +187,23 @@ def cross_attn(q, k_ctx, v_ctx, o, ctx_lens, softmax_scale=None,
     _check(lib().wan_cross_attn(_ptr(q), _ptr(k_ctx), _ptr(v_ctx), _ptr(o),
                                 lens, B, Lq, Lk, H, D, softmax_scale,
                                 _stream(stream)), "wan_cross_attn")
+
+
+def block_causal_attn(q, k, v, o, chunk_tokens, q_offset=0,
+                      softmax_scale=None, stream=None):
+    """Chunk-wise causal attention: query a = q_offset + i sees keys
+    j < (a // chunk_tokens + 1) * chunk_tokens (and j < Lk)."""
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o)):
+        _bf16_bl(t, name)
+    B, Lq, H, D = q.shape
+    Lk = k.shape[1]
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(D)
+    _check(lib().wan_block_causal_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(o),
+                                       B, Lq, Lk, H, D, int(chunk_tokens),
+                                       int(q_offset), softmax_scale,
+                                       _stream(stream)),
+           "wan_block_causal_attn")
 
 
 def fm_step(x, v_cond, v_uncond, guide, sigma, sigma_next, stream=None):
