@@ -45,6 +45,8 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-hbm", action="store_true",
                    help="skip the HBM-bound kernel rooflines")
+    p.add_argument("--no-causal", action="store_true",
+                   help="skip the block-causal attention measurement")
     p.add_argument("--hbm-elems", type=int, default=1 << 28,
                    help="fp32 elements per buffer of the fm_step roofline")
     p.add_argument("--cpu-rows", type=int, default=4096,
@@ -294,6 +296,57 @@ def hbm_rooflines(dev, g, L, H, n_lat, peak_gbs, n=1 << 28, reps=20):
     return out
 
 
+def causal_rooflines(dev, peak_tflops, reps=5):
+    """Block-causal (Self Forcing chunk) attention at 480p-165f: 42 x 30 x
+    52 = 65,520 tokens, 40 heads, chunks of 3 latent frames (4,680 tokens).
+    Times the full-sequence call and the KV-cache step of the last chunk
+    (4,680 queries against all 65,520 keys).  FLOPs count only visible keys:
+    4 * 128 * heads * sum over queries of the key limit."""
+    import numpy as np
+    import torch
+
+    from video_diffusion_transformer_self_b200 import wan
+    from video_diffusion_transformer_self_b200.workloads import WORKLOADS
+
+    w = WORKLOADS[4]
+    _, g = wan.token_grid(w.frames, w.height, w.width)
+    L, H = g.F * g.H * g.W, w.heads
+    chunk = 3 * g.H * g.W
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(5151)
+    q = torch.randn(1, L, H, 128, device=dev, generator=gen).to(torch.bfloat16)
+    k = torch.randn(1, L, H, 128, device=dev, generator=gen).to(torch.bfloat16)
+    v = torch.randn(1, L, H, 128, device=dev, generator=gen).to(torch.bfloat16)
+    o = torch.empty_like(q)
+
+    def visible(lq, off):
+        a = off + np.arange(lq, dtype=np.int64)
+        return float(np.minimum(L, (a // chunk + 1) * chunk).sum())
+
+    out = {"workload": "480p-165f", "tokens": L, "heads": H,
+           "chunk_tokens": chunk}
+    for name, qq, off in (("full_sequence", q, 0),
+                          ("kv_cache_last_chunk",
+                           q[:, L - chunk:].contiguous(), L - chunk)):
+        oo = o[:, :qq.shape[1]] if off else o
+        for _ in range(2):
+            wan.block_causal_attn(qq, k, v, oo, chunk, off)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(reps):
+            wan.block_causal_attn(qq, k, v, oo, chunk, off)
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / reps
+        fl = 4.0 * 128 * H * visible(qq.shape[1], off)
+        out[name] = {"ms": ms, "tflops": fl / (ms / 1e3) / 1e12,
+                     "frac_of_sustained_peak": fl / (ms / 1e3) / 1e12
+                     / peak_tflops}
+    return out
+
+
 def run_wan(args, w, rank, world, local_rank):
     import numpy as np
     import torch
@@ -525,6 +578,8 @@ def run_wan(args, w, rank, world, local_rank):
         line["hbm_kernels"] = hbm_rooflines(
             dev, g, L, H, n_lat, float(pk.get("hbm_gbs", 6650.0)),
             n=args.hbm_elems)
+    if not args.no_causal and world == 1:
+        line["block_causal"] = causal_rooflines(dev, peak)
     if not args.no_cpu_baseline and world == 1:
         dt, fl, text = cpu_oracle_sample(w, args.cpu_rows)
         line["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": "TFLOP/s",
