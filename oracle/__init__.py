@@ -22,7 +22,9 @@ Modules:
 * ``rope``      -- 3D rotary position embedding (t/h/w bands);
 * ``attention`` -- softmax self-attention and length-masked cross-attention;
 * ``schedule``  -- shifted sigma schedule and timestep scale;
-* ``step``      -- classifier-free-guidance combine and Euler flow step.
+* ``step``      -- classifier-free-guidance combine and Euler flow step;
+* ``block``     -- AdaLN modulate, QK-Norm + RoPE, gated residual around the
+  attention.
 
 Pins (tests/test_oracle_*.py) tie each function to numbers the pages print,
 closed forms and brute force.  The one part the pages do not fix numerically
@@ -32,4 +34,4 @@ state (translation invariance of q.k, identity at the origin, norm
 preservation); the readings taken are listed in ``rope``'s docstring.
 """
 
-from . import grid, rope, attention, schedule, step  # noqa: F401
+from . import grid, rope, attention, schedule, step, block  # noqa: F401
