@@ -273,7 +273,46 @@ def hbm_rooflines(dev, g, L, H, n_lat, peak_gbs, n=1 << 28, reps=20):
     out["rope3d_qk"] = {"tokens": L, "heads": H, "bytes_per_call": nbytes,
                         "ms": ms, "achieved_gbs": gbs, "peak_gbs": peak_gbs,
                         "frac": gbs / peak_gbs}
+    # QK-Norm + RoPE on the same Q / K (same traffic as the RoPE pass)
+    wq = torch.randn(H * 128, device=dev, generator=gen)
+    wk = torch.randn(H * 128, device=dev, generator=gen)
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    ms = timed(lambda: wan.qk_norm_rope(q, k, wq, wk, g, table))
+    out["qk_norm_rope"] = {"bytes_per_call": nbytes, "ms": ms,
+                           "achieved_gbs": nbytes / (ms / 1e3) / 1e9,
+                           "peak_gbs": peak_gbs,
+                           "frac": nbytes / (ms / 1e3) / 1e9 / peak_gbs}
     del q, k
+    # AdaLN modulate and gated residual on the fp32 residual stream
+    D = H * 128
+    x = torch.randn(1, L, D, device=dev, generator=gen)
+    sh = torch.randn(1, D, device=dev, generator=gen)
+    sc = torch.randn(1, D, device=dev, generator=gen)
+    yb = torch.empty(1, L, D, device=dev, dtype=torch.bfloat16)
+    ms = timed(lambda: wan.adaln_modulate(x, sh, sc, yb))
+    nb = x.numel() * 6
+    out["adaln_modulate"] = {"bytes_per_call": nb, "ms": ms,
+                             "achieved_gbs": nb / (ms / 1e3) / 1e9,
+                             "peak_gbs": peak_gbs,
+                             "frac": nb / (ms / 1e3) / 1e9 / peak_gbs}
+    ms = timed(lambda: wan.gated_residual(x, yb, sh))
+    nb = x.numel() * 10
+    out["gated_residual"] = {"bytes_per_call": nb, "ms": ms,
+                             "achieved_gbs": nb / (ms / 1e3) / 1e9,
+                             "peak_gbs": peak_gbs,
+                             "frac": nb / (ms / 1e3) / 1e9 / peak_gbs}
+    del x, yb
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
     xl = torch.randn(n_lat, device=dev, generator=gen)
     cl = torch.randn(n_lat, device=dev, generator=gen)

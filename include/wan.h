@@ -145,6 +145,30 @@ int wan_block_causal_attn(const void* q, const void* k, const void* v,
                           int head_dim, int chunk_tokens, int q_offset,
                           float softmax_scale, void* s);
 
+/* ---------------------------------------- block prologue and epilogue --
+ * Wan2.2 source reading, ch. 4, section "Full forward of one block": the
+ * self-attention input is norm1(x) * (1 + e[1]) + e[0] and the block output
+ * x + y * e[2] (fp32 autocast); section "3D RoPE": q and k each pass an
+ * RMSNorm (QK-Norm) after their linear layers, before the rotation.
+ *
+ * wan_adaln_modulate: out[b,l,:] = LN(x[b,l,:]) * (1 + scale[b,:])
+ *   + shift[b,:], LN over D without affine weights, variance eps.  x fp32
+ *   [B, L, D]; shift, scale fp32 [B, D]; out bf16 [B, L, D].  D % 4 == 0,
+ *   D <= 8192, all pointers 16-byte aligned.
+ * wan_qk_norm_rope: in place on q and k ([B, L, heads, 128] bf16, either may
+ *   be NULL): t <- rope3d(t / sqrt(mean_{heads*128}(t^2) + eps) * w), the
+ *   mean over all heads of a token, w fp32 [heads * 128] (wq for q, wk for
+ *   k), then the 3D RoPE of grid g with the wan_rope3d_table layout.
+ * wan_gated_residual: x[b,l,:] += y[b,l,:] * gate[b,:]; x fp32 [B, L, D],
+ *   y bf16 [B, L, D] (8-byte aligned), gate fp32 [B, D].  D % 4 == 0.       */
+int wan_adaln_modulate(const float* x, const float* shift, const float* scale,
+                       void* out, int B, int L, int D, float eps, void* s);
+int wan_qk_norm_rope(void* q, void* k, const float* wq, const float* wk,
+                     int B, wan_grid_t g, int heads, int head_dim,
+                     const void* d_table, float eps, void* s);
+int wan_gated_residual(float* x, const void* y, const float* gate, int B,
+                       int L, int D, void* s);
+
 /* ------------------------------------------------------------- sampler --
  * Wan2.2 source reading, ch. 5, section "shift": the points are laid
  * uniformly and mapped by sigma = shift*s / (1 + (shift-1)*s); ch. 1

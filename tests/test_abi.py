@@ -146,3 +146,19 @@ def test_argument_checks_without_device(lib):
                                    None) == wan.WAN_EINVAL
     assert L.wan_block_causal_attn(odd, p, p, o, 1, 10, 20, 2, 128, 5, 0, 0.1,
                                    None) == wan.WAN_EALIGN
+    assert L.wan_adaln_modulate(p, p, p, o, 1, 4, 6, 1e-6, None) \
+        == wan.WAN_EINVAL  # D % 4
+    assert L.wan_adaln_modulate(p, p, p, o, 1, 4, 8196 + 4, 1e-6, None) \
+        == wan.WAN_EINVAL  # D too large
+    assert L.wan_adaln_modulate(p, p, p, o, 1, 4, 8, 0.0, None) \
+        == wan.WAN_EINVAL  # eps
+    assert L.wan_adaln_modulate(odd, p, p, o, 1, 4, 8, 1e-6, None) \
+        == wan.WAN_EALIGN
+    assert L.wan_qk_norm_rope(p, None, None, None, 1, g, 2, 128, p, 1e-6,
+                              None) == wan.WAN_EINVAL  # q without weight
+    assert L.wan_qk_norm_rope(None, None, p, p, 1, g, 2, 128, p, 1e-6,
+                              None) == wan.WAN_EINVAL
+    assert L.wan_qk_norm_rope(p, p, p, p, 1, g, 2, 128, p, 1e-6, None) \
+        == wan.WAN_EINVAL  # q aliases k
+    assert L.wan_gated_residual(p, p, p, 1, 4, 6, None) == wan.WAN_EINVAL
+    assert L.wan_gated_residual(odd, p, p, 1, 4, 8, None) == wan.WAN_EALIGN

@@ -57,6 +57,11 @@ _SIGNATURES = {
                             _I, _I, _I, _I, _I, ctypes.c_float, _P]),
     "wan_block_causal_attn": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I,
                                    _I, ctypes.c_float, _P]),
+    "wan_adaln_modulate": (_I, [_P, _P, _P, _P, _I, _I, _I, ctypes.c_float,
+                                _P]),
+    "wan_qk_norm_rope": (_I, [_P, _P, _P, _P, _I, Grid, _I, _I, _P,
+                              ctypes.c_float, _P]),
+    "wan_gated_residual": (_I, [_P, _P, _P, _I, _I, _I, _P]),
     "wan_fm_sigmas": (_I, [_I, ctypes.c_double, ctypes.c_double,
                            ctypes.POINTER(ctypes.c_double)]),
     "wan_fm_step": (_I, [_P, _P, _P, ctypes.c_float, ctypes.c_int64,
@@ -204,6 +209,47 @@ def block_causal_attn(q, k, v, o, chunk_tokens, q_offset=0,
                                        int(q_offset), softmax_scale,
                                        _stream(stream)),
            "wan_block_causal_attn")
+
+
+def _f32(t, name):
+    import torch
+    if t.dtype != torch.float32 or not t.is_contiguous() or not t.is_cuda:
+        raise ValueError("%s must be a contiguous CUDA fp32 tensor" % name)
+
+
+def adaln_modulate(x, shift, scale, out, eps=1e-6, stream=None):
+    """out = LayerNorm(x) * (1 + scale[b]) + shift[b]; x fp32 [B, L, D]."""
+    import torch
+    for name, t in (("x", x), ("shift", shift), ("scale", scale)):
+        _f32(t, name)
+    if out.dtype != torch.bfloat16 or not out.is_contiguous():
+        raise ValueError("out must be a contiguous bf16 tensor")
+    B, L, D = x.shape
+    _check(lib().wan_adaln_modulate(_ptr(x), _ptr(shift), _ptr(scale),
+                                    _ptr(out), B, L, D, eps,
+                                    _stream(stream)), "wan_adaln_modulate")
+
+
+def qk_norm_rope(q, k, wq, wk, g, table, eps=1e-6, stream=None):
+    """In place: t = rope3d(RMSNorm_{heads*128}(t) * w) for t in (q, k)."""
+    t = q if q is not None else k
+    _bf16_bl(t, "q/k")
+    for name, w in (("wq", wq), ("wk", wk)):
+        if w is not None:
+            _f32(w, name)
+    _check(lib().wan_qk_norm_rope(_ptr(q), _ptr(k), _ptr(wq), _ptr(wk),
+                                  t.shape[0], g, t.shape[2], t.shape[3],
+                                  _ptr(table), eps, _stream(stream)),
+           "wan_qk_norm_rope")
+
+
+def gated_residual(x, y, gate, stream=None):
+    """x += y * gate[b]; x fp32 [B, L, D], y bf16 [B, L, D], gate [B, D]."""
+    _f32(x, "x")
+    _f32(gate, "gate")
+    B, L, D = x.shape
+    _check(lib().wan_gated_residual(_ptr(x), _ptr(y), _ptr(gate), B, L, D,
+                                    _stream(stream)), "wan_gated_residual")
 
 
 def fm_step(x, v_cond, v_uncond, guide, sigma, sigma_next, stream=None):
