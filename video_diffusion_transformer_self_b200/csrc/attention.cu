@@ -15,16 +15,21 @@
 // Warp roles (384 threads, registers rebalanced with setmaxnreg):
 //   warps 0-3 / 4-7  softmax of tile 0 / tile 1: thread r owns query row r
 //              (TMEM lane r).  Reads the 128x128 fp32 score tile from TMEM,
-//              keeps the running row max (log2 units) and sum, writes P
-//              (bf16) back into TMEM over its scores, rescales O in TMEM when
-//              the max grows by more than 2^8 (exact after the final O / l),
-//              and writes the bf16 epilogue.  A quarter of the exponentials
+//              keeps the running row max (log2 units) and sum, rescales O
+//              in TMEM when the max grows by more than 2^8 (exact after the
+//              final O / l), writes P (bf16) back into TMEM over its
+//              scores, and writes the bf16 epilogue.  A quarter of the exponentials
 //              run on the FMA pipe (exp2_fma2) to offload the MUFU unit.
 //   warp 8     TMA producer: the two Q tiles once, then K (3-stage ring) and
 //              V (2-stage ring).
 //   warp 9     MMA issuer (one lane): S_t = Q_t K^T (both operands K-major in
 //              smem) and O_t += P_t V (P from TMEM, V MN-major in smem), in
-//              the order PV_0(j-1), S_0(j), PV_1(j-1), S_1(j).
+//              the order PV_0(j-1), S_0(j), PV_1(j-1), S_1(j).  Measured:
+//              tcgen05.mma issue slows from 64 to 89 cycles per MMA while
+//              FMA work fills this warp's sub-partition (MUFU or integer
+//              work there, or FMA work on another sub-partition, does not
+//              slow it), so the 16 MMAs that follow each softmax sit on the
+//              tile's critical path.  A second issuer warp measured slower.
 //   warps 10-11  RoPE variant: rotate the Q tiles and every K tile in shared
 //              memory before the tensor cores read them.
 // Tensor memory (512 columns): S/P of tile 0 at 0, of tile 1 at 128, O of
@@ -60,6 +65,13 @@ constexpr int kOtherRegs = 88;               // warps 8-11
 constexpr int kRopeThreads = 64;             // warps 10-11
 constexpr int MAX_CROSS_BATCH = 512;
 constexpr float RESCALE_LOG2 = 8.0f;         // rescale O when max grows > 2^8
+// P of a tile can be published in NPART key ranges so that P V on the
+// first keys overlaps the exponentials of the rest.  Measured on B200 at
+// 32,760 and 75,600 tokens: 2 parts 6% and 4 parts 20% slower than 1 (each
+// publication waits for the warp's TMEM stores), so P is published whole.
+constexpr int NPART = 1;
+constexpr int KPP = BN / 16 / NPART;         // P V K-steps per part
+static_assert(BN % (32 * NPART) == 0, "parts of whole 32-key chunks");
 // Pairs (2e, 2e+1) with (e & 7) < kEmuPer8 take the FMA-pipe exponential.
 constexpr int kEmuPer8 = 2;
 
@@ -88,8 +100,8 @@ enum : int {
   B_VFULL = B_KEMPTY + NSK,
   B_VEMPTY = B_VFULL + NSV,
   B_SFULL = B_VEMPTY + NSV,  // per tile
-  B_PFULL = B_SFULL + QT,    // per tile, one arrival per softmax warp
-  B_OFINAL = B_PFULL + QT,   // per tile, the last PV only (single phase)
+  B_PPART = B_SFULL + QT,    // per tile and part, one arrival per warp
+  B_OFINAL = B_PPART + QT * NPART,  // per tile, last PV only (single phase)
   B_DRAIN = B_OFINAL + QT,
   NBAR = B_DRAIN + 1
 };
@@ -251,14 +263,16 @@ __device__ __forceinline__ float rowmax(const float* s) {
 // exponential for part of the pairs (never for a masked block, whose -inf
 // entries must give exact zeros).
 template <bool kEmu>
-__device__ __forceinline__ float exp_store_row(const float* s, float c2,
-                                               float m, uint32_t pcol) {
+__device__ __forceinline__ void exp_store_chunks(const float* s, float c2,
+                                                 float m, uint32_t pcol,
+                                                 float2 (&acc)[4], int c0,
+                                                 int c1) {
+  // Chunks [c0, c1) of 32 keys (constants after unrolling): p = 2^(s c2 - m), packed to bf16 pairs into
+  // the tile's P columns (16 per chunk), p summed into acc in fp32.
   const float2 c22 = make_float2(c2, c2);
   const float2 nm2 = make_float2(-m, -m);
-  float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                   make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-  for (int c = 0; c < 4; ++c) {
+  for (int c = c0; c < c1; ++c) {
     uint32_t pk[16];
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
@@ -277,8 +291,6 @@ __device__ __forceinline__ float exp_store_row(const float* s, float c2,
     }
     tmem_st16(pcol + c * 16, pk);
   }
-  const float2 t = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
-  return t.x + t.y;
 }
 
 template <int kRope>
@@ -330,7 +342,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int t = 0; t < QT; ++t) {
       mbar_init(&bar[B_SFULL + t], 1);
-      mbar_init(&bar[B_PFULL + t], 4);
+      for (int q = 0; q < NPART; ++q) mbar_init(&bar[B_PPART + t * NPART + q], 4);
       mbar_init(&bar[B_OFINAL + t], 1);
     }
     mbar_init(&bar[B_DRAIN], 1);
@@ -426,19 +438,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
       };
-      // O_t += P_t(i) V(i).
-      auto issue_pv = [&](int t, int i) {
+      // O_t += P_t(i) V(i) over the keys of P part `part`.
+      auto issue_pv_part = [&](int t, int i, int part) {
         const uint64_t b0 = dv + (((i % NSV) * TILE) >> 4);
         const uint32_t d = tmem + TM_O + t * 128;
         const uint32_t a = tmem + t * 128;
-        const uint32_t acc = i > 0 ? 1u : 0u;
         if (leader) {
           // B = V[16k .. 16k+15][0..127]: MN-major, 8-key groups 1024 B
           // apart (SBO), the two 64-channel halves 16 KB apart (LBO).
-          umma_ts(d, a, b0, IDESC_PV, acc);
 #pragma unroll
-          for (int k = 1; k < BN / 16; ++k)
-            umma_ts(d, a + k * 8, b0 + ((k * 2048) >> 4), IDESC_PV, 1u);
+          for (int kk = 0; kk < KPP; ++kk) {
+            const int k = part * KPP + kk;
+            umma_ts(d, a + k * 8, b0 + ((k * 2048) >> 4), IDESC_PV,
+                    (i > 0 || k > 0) ? 1u : 0u);
+          }
         }
         __syncwarp();
       };
@@ -447,18 +460,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (leader) umma_commit(b);
         __syncwarp();
       };
-      // Waits for P_0(i) and V(i), clears text-padding rows of V(i).
-      // V(i) is waited for first: it does not depend on the softmax, so the
-      // issue of PV_0(i) follows P_0(i) as closely as possible.
-      auto ready_pv0 = [&](int i) -> bool {
+      // Waits for V(i) and clears its text-padding rows: they may hold
+      // anything (NaN included), and P is 0 there but 0 * NaN is not.
+      auto ready_v = [&](int i) -> bool {
         if (!wait_warp(&bar[B_VFULL + i % NSV], (i / NSV) & 1, abort_flag,
                        status))
           return false;
-        if (!wait_warp(&bar[B_PFULL + 0], i & 1, abort_flag, status))
-          return false;
         if (args.cross && kv_len < (i + 1) * BN) {
-          // Text padding rows may hold anything (NaN included): P is 0 there
-          // but 0 * NaN is not, so clear those V rows before the MMA.
           const int first = kv_len - i * BN;
           uint8_t* vt = sV + (i % NSV) * TILE;
           for (int idx = lane; idx < (BN - first) * 16; idx += 32) {
@@ -470,7 +478,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           fence_proxy_async_smem();
           __syncwarp();
         }
-        tc_fence_after();
+        return true;
+      };
+      // O_t += P_t(i) V(i), each part issued as soon as the softmax warps
+      // have published it.
+      auto pv = [&](int t, int i) -> bool {
+        for (int part = 0; part < NPART; ++part) {
+          if (!wait_warp(&bar[B_PPART + t * NPART + part], i & 1, abort_flag,
+                         status))
+            return false;
+          tc_fence_after();
+          issue_pv_part(t, i, part);
+        }
         return true;
       };
       bool ok = wait_warp(&bar[kRope ? B_QREADY : B_QFULL], 0, abort_flag,
@@ -478,9 +497,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < nblk && ok; ++j) {
         const int sk = j % NSK;
         if (j > 0) {
-          ok = ready_pv0(j - 1);
+          ok = ready_v(j - 1) && pv(0, j - 1);
           if (!ok) break;
-          issue_pv(0, j - 1);
         }
         ok = wait_warp(&bar[(kRope ? B_KREADY : B_KFULL) + sk], (j / NSK) & 1,
                        abort_flag, status);
@@ -488,10 +506,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         issue_s(0, j);
         if (j > 0) {
-          ok = wait_warp(&bar[B_PFULL + 1], (j - 1) & 1, abort_flag, status);
+          ok = pv(1, j - 1);
           if (!ok) break;
-          tc_fence_after();
-          issue_pv(1, j - 1);
           commit(&bar[B_VEMPTY + (j - 1) % NSV]);
         }
         issue_s(1, j);
@@ -499,15 +515,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (ok) {
         const int i = nblk - 1;
-        ok = ready_pv0(i);
+        ok = ready_v(i) && pv(0, i);
         if (ok) {
-          issue_pv(0, i);
           commit(&bar[B_OFINAL + 0]);
-          ok = wait_warp(&bar[B_PFULL + 1], i & 1, abort_flag, status);
+          ok = pv(1, i);
         }
         if (ok) {
-          tc_fence_after();
-          issue_pv(1, i);
           commit(&bar[B_OFINAL + 1]);
           commit(&bar[B_VEMPTY + i % NSV]);
         }
@@ -574,23 +587,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < BN; ++c)
           if (c >= lim) s[c] = -INFINITY;
       }
-      float sum;
+      const float mx = (masked ? rowmax_masked<BN>(s) : rowmax<BN>(s)) * c2;
       if (j == 0) {
-        m_run = (masked ? rowmax_masked<BN>(s) : rowmax<BN>(s)) * c2;
-        sum = masked ? exp_store_row<false>(s, c2, m_run, s_col)
-                     : exp_store_row<true>(s, c2, m_run, s_col);
+        m_run = mx;
       } else {
-        // Exponentiate against the running max right away and find this
-        // block's max alongside: with no rescale the exponents stay <= 8
-        // (p <= 256, exact after the final O / l).  Only when some row's max
-        // grew by more than 2^8 is O rescaled and P formed again.
-        const float mx = (masked ? rowmax_masked<BN>(s) : rowmax<BN>(s)) * c2;
-        sum = masked ? exp_store_row<false>(s, c2, m_run, s_col)
-                     : exp_store_row<true>(s, c2, m_run, s_col);
+        // Keep the running max unless some row's max grew by more than 2^8:
+        // exponents then stay <= 8 (p <= 256, exact after the final O / l).
+        // Otherwise rescale O in TMEM first.  S_t(j) complete implies
+        // PV_t(j-1) complete (issued before it), so O holds exactly blocks
+        // 0..j-1 here; the first part's arrival orders these stores before
+        // PV_t(j).
         const bool need = mx > m_run + RESCALE_LOG2;
         if (__any_sync(0xffffffffu, need)) {
-          // S_t(j) complete implies PV_t(j-1) complete (issued before it),
-          // so O holds exactly blocks 0..j-1 here.
           const float m_new = need ? mx : m_run;
           const float alpha = ex2(m_run - m_new);
 #pragma unroll
@@ -610,16 +618,31 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           l_run *= alpha;
           m_run = m_new;
-          tmem_st_wait();  // the first P stores land before they are redone
-          sum = masked ? exp_store_row<false>(s, c2, m_run, s_col)
-                       : exp_store_row<true>(s, c2, m_run, s_col);
         }
       }
-      l_run += sum;
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar[B_PFULL + t]);
+      float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                       make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+      // Publish P part by part: the MMA issuer starts P V on the first keys
+      // while the rest are exponentiated.
+      auto publish = [&](int part) {
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[B_PPART + t * NPART + part]);
+      };
+      constexpr int CPP = BN / 32 / NPART;  // 32-key chunks per part
+#pragma unroll
+      for (int part = 0; part < NPART; ++part) {
+        if (masked)
+          exp_store_chunks<false>(s, c2, m_run, s_col, acc, part * CPP,
+                                  (part + 1) * CPP);
+        else
+          exp_store_chunks<true>(s, c2, m_run, s_col, acc, part * CPP,
+                                 (part + 1) * CPP);
+        publish(part);
+      }
+      const float2 tsum = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
+      l_run += tsum.x + tsum.y;
     }
     if (ok) ok = wait_warp(&bar[B_OFINAL + t], 0, abort_flag, status);
     if (ok) {
