@@ -24,7 +24,10 @@ Modules:
 * ``schedule``  -- shifted sigma schedule and timestep scale;
 * ``step``      -- classifier-free-guidance combine and Euler flow step;
 * ``block``     -- AdaLN modulate, QK-Norm + RoPE, gated residual around the
-  attention.
+  attention;
+* ``unipc``     -- the UniPC order-2 predictor-corrector sampler step (the
+  pages give no coefficients: written from the published UniPC order
+  conditions, pinned by exactness and convergence order).
 
 Pins (tests/test_oracle_*.py) tie each function to numbers the pages print,
 closed forms and brute force.  The one part the pages do not fix numerically
@@ -34,4 +37,4 @@ state (translation invariance of q.k, identity at the origin, norm
 preservation); the readings taken are listed in ``rope``'s docstring.
 """
 
-from . import grid, rope, attention, schedule, step, block  # noqa: F401
+from . import grid, rope, attention, schedule, step, block, unipc  # noqa: F401,E501
