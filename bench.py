@@ -225,11 +225,12 @@ def job_throughput(world, flops_per_step, steps, max_ms):
 
 
 def hbm_rooflines(dev, g, L, H, n_lat, peak_gbs, n=1 << 28, reps=20):
-    """Achieved bandwidth of the two HBM-bound kernels, timed alone with CUDA
-    events: the fused CFG + Euler step on n-element fp32 buffers (default
-    2^28: 4 GiB of traffic per call, far above L2) and the RoPE pass on the
-    workload's Q and K; plus the step on the workload's own latent, timed
-    cold (L2 flushed by a 512 MiB write before every call)."""
+    """Achieved bandwidth of the HBM-bound kernels, timed alone with CUDA
+    events: the fused CFG + Euler step and the fused UniPC stop on n-element
+    fp32 buffers (default 2^28: 4 GiB / 9 GiB of traffic per call, far above
+    L2), the RoPE, QK-Norm + RoPE, AdaLN and gated-residual passes on the
+    workload's tensors; plus the Euler step on the workload's own latent,
+    timed cold (L2 flushed by a 512 MiB write before every call)."""
     import torch
 
     from video_diffusion_transformer_self_b200 import wan
@@ -255,7 +256,28 @@ def hbm_rooflines(dev, g, L, H, n_lat, peak_gbs, n=1 << 28, reps=20):
     out["fm_step_cfg"] = {"elements": n, "bytes_per_call": 16 * n,
                           "ms": ms, "achieved_gbs": gbs, "peak_gbs": peak_gbs,
                           "frac": gbs / peak_gbs}
-    del x, c, u
+    # UniPC stop 20 of the 40-step shift-12 schedule: CFG, order-2 corrector
+    # and predictor; 36 B per element (x, x_corr, m_(i-1), m_(i-2), v_cond,
+    # v_uncond read; x, x_corr, m_i written, m_i over m_(i-2)).
+    xc = torch.randn(n, device=dev, generator=gen)
+    m1 = torch.randn(n, device=dev, generator=gen)
+    m2 = torch.randn(n, device=dev, generator=gen)
+    sig = wan.fm_sigmas(40, 12.0)
+    for _ in range(3):
+        wan.unipc_step(x, xc, m1, m2, m2, c, u, 4.0, sig, 20)
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(reps):
+        wan.unipc_step(x, xc, m1, m2, m2, c, u, 4.0, sig, 20)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    gbs = 36.0 * n / (ms / 1e3) / 1e9
+    out["unipc_step_cfg"] = {"elements": n, "bytes_per_call": 36 * n,
+                             "stop": 20, "corrector_order": 2,
+                             "ms": ms, "achieved_gbs": gbs,
+                             "peak_gbs": peak_gbs, "frac": gbs / peak_gbs}
+    del x, c, u, xc, m1, m2
     q = torch.randn(1, L, H, 128, device=dev, generator=gen).to(torch.bfloat16)
     k = torch.randn(1, L, H, 128, device=dev, generator=gen).to(torch.bfloat16)
     table = wan.rope3d_table(g)

@@ -191,6 +191,49 @@ int wan_fm_step(float* x, const float* v_cond, const float* v_uncond,
                 float guide, int64_t n, double sigma, double sigma_next,
                 void* s);
 
+/* -------------------------------------------------------------- UniPC ---
+ * Wan2.2 source reading, ch. 5 "UniPC": the default sampler is a multistep
+ * predictor-corrector of order 2; the predictor extrapolates the trend of
+ * the last two model outputs, the corrector redoes the step just taken with
+ * the new output (no extra forward).  Ch. 1: x = (1 - sigma) x0 + sigma
+ * noise, clean estimate m = x - sigma v.  The pages give no coefficients:
+ * they follow the published UniPC order conditions (data prediction,
+ * lambda = log((1 - sigma) / sigma), coefficients solved exactly); the step
+ * to sigma = 0 is first order and an earlier stop at sigma = 1 is dropped.
+ *
+ * wan_unipc_coeffs: host, fp64.  Folded coefficients of stop i (0 <= i <
+ * n_steps) of the schedule sigmas[0 .. n_steps] (strictly decreasing, in
+ * [0, 1], sigmas[n_steps] >= 0):
+ *   m_i   = x~_i - sigma * v
+ *   x^c_i = cx x^c_(i-1) + cm1 m_(i-1) + cm2 m_(i-2) + cm m_i  (corr_order
+ *           1 or 2: differences used, the new point included; corr_order 0
+ *           at i == 0, where x^c_0 = x~_0)
+ *   x~_(i+1) = px x^c_i + pm m_i + pm1 m_(i-1)  (pred_order 1 or 2).
+ *   WAN_EINVAL for a bad schedule or index.
+ *
+ * wan_unipc_step: device, fp32, n elements, one fused pass:
+ *   v = v_cond, or v_uncond + guide * (v_cond - v_uncond) if v_uncond;
+ *   x      in: x~_i      out: x~_(i+1)
+ *   x_corr in: x^c_(i-1) (not read at i == 0)   out: x^c_i
+ *   m_prev1 = m_(i-1) (read if i >= 1), m_prev2 = m_(i-2) (read if
+ *   corr_order == 2), m_out receives m_i and may alias m_prev2 (a caller
+ *   keeps two buffers and swaps them); no other pointers may alias.  All
+ *   16-byte aligned (WAN_EALIGN); coefficients rounded once to fp32.       */
+typedef struct {
+  double sigma;
+  double cx, cm1, cm2, cm;
+  double px, pm, pm1;
+  int32_t pred_order;
+  int32_t corr_order;
+} wan_unipc_coef_t;
+
+int wan_unipc_coeffs(const double* sigmas, int n_steps, int i,
+                     wan_unipc_coef_t* out);
+int wan_unipc_step(float* x, float* x_corr, const float* m_prev1,
+                   const float* m_prev2, float* m_out, const float* v_cond,
+                   const float* v_uncond, float guide, int64_t n,
+                   const double* sigmas, int n_steps, int i, void* s);
+
 /* ------------------------------------------------------------- status ---
  * Reads (and, if clear != 0, resets) the device status word of the current
  * device: 0 or WAN_ETIMEOUT.  Synchronous (waits for the device).          */

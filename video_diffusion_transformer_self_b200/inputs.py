@@ -14,6 +14,7 @@ import torch
 ROLE = {
     "q": 0, "k": 1, "v": 2, "k_ctx": 3, "v_ctx": 4, "lens": 5,
     "x": 6, "v_cond": 7, "v_uncond": 8, "x0": 9, "rows": 10,
+    "x_corr": 11, "m_prev1": 12, "m_prev2": 13,
 }
 
 

@@ -40,8 +40,22 @@ class Grid(ctypes.Structure):
         return "Grid(%d, %d, %d)" % (self.F, self.H, self.W)
 
 
+class UniPCCoef(ctypes.Structure):
+    """wan_unipc_coef_t: folded coefficients of one UniPC stop."""
+    _fields_ = [("sigma", ctypes.c_double), ("cx", ctypes.c_double),
+                ("cm1", ctypes.c_double), ("cm2", ctypes.c_double),
+                ("cm", ctypes.c_double), ("px", ctypes.c_double),
+                ("pm", ctypes.c_double), ("pm1", ctypes.c_double),
+                ("pred_order", ctypes.c_int32),
+                ("corr_order", ctypes.c_int32)]
+
+    def as_dict(self):
+        return {name: getattr(self, name) for name, _ in self._fields_}
+
+
 _P = ctypes.c_void_p
 _I = ctypes.c_int
+_D = ctypes.POINTER(ctypes.c_double)
 _SIGNATURES = {
     "wan_status_string": (ctypes.c_char_p, [_I]),
     "wan_version": (_I, []),
@@ -66,6 +80,9 @@ _SIGNATURES = {
                            ctypes.POINTER(ctypes.c_double)]),
     "wan_fm_step": (_I, [_P, _P, _P, ctypes.c_float, ctypes.c_int64,
                          ctypes.c_double, ctypes.c_double, _P]),
+    "wan_unipc_coeffs": (_I, [_D, _I, _I, ctypes.POINTER(UniPCCoef)]),
+    "wan_unipc_step": (_I, [_P, _P, _P, _P, _P, _P, _P, ctypes.c_float,
+                            ctypes.c_int64, _D, _I, _I, _P]),
     "wan_device_status": (_I, [_I]),
 }
 
@@ -261,6 +278,40 @@ def fm_step(x, v_cond, v_uncond, guide, sigma, sigma_next, stream=None):
     _check(lib().wan_fm_step(_ptr(x), _ptr(v_cond), _ptr(v_uncond), guide,
                              x.numel(), sigma, sigma_next, _stream(stream)),
            "wan_fm_step")
+
+
+def _sigma_array(sigmas):
+    arr = (ctypes.c_double * len(sigmas))(*[float(x) for x in sigmas])
+    return arr, len(sigmas) - 1
+
+
+def unipc_coeffs(sigmas, i):
+    """Folded UniPC coefficients of stop i (dict of wan_unipc_coef_t)."""
+    arr, n = _sigma_array(sigmas)
+    out = UniPCCoef()
+    _check(lib().wan_unipc_coeffs(arr, n, int(i), ctypes.byref(out)),
+           "wan_unipc_coeffs")
+    return out.as_dict()
+
+
+def unipc_step(x, x_corr, m_prev1, m_prev2, m_out, v_cond, v_uncond, guide,
+               sigmas, i, stream=None):
+    """One fused UniPC stop (see include/wan.h): x and x_corr in place,
+    m_i into m_out (which may be the m_prev2 buffer)."""
+    import torch
+    for name, t in (("x", x), ("x_corr", x_corr), ("m_out", m_out),
+                    ("v_cond", v_cond), ("v_uncond", v_uncond),
+                    ("m_prev1", m_prev1), ("m_prev2", m_prev2)):
+        if t is not None and (t.dtype != torch.float32 or not t.is_cuda
+                              or not t.is_contiguous()
+                              or t.numel() != x.numel()):
+            raise ValueError("%s must be a contiguous CUDA fp32 tensor of "
+                             "x's size" % name)
+    arr, n = _sigma_array(sigmas)
+    _check(lib().wan_unipc_step(_ptr(x), _ptr(x_corr), _ptr(m_prev1),
+                                _ptr(m_prev2), _ptr(m_out), _ptr(v_cond),
+                                _ptr(v_uncond), guide, x.numel(), arr, n,
+                                int(i), _stream(stream)), "wan_unipc_step")
 
 
 def device_status(clear=True):
