@@ -38,8 +38,11 @@ def test_adaln_modulate(B, L, D):
     _bf16_bound(out.double().cpu().numpy(), want, 1e-5 * (1 + np.abs(want)))
 
 
+# heads <= 40 take the register-resident kernel, more heads the two-pass one
 @pytest.mark.parametrize("grid,B,H", [((2, 4, 4), 1, 2), ((3, 7, 13), 2, 12),
-                                      ((5, 30, 52), 1, 40)])
+                                      ((5, 30, 52), 1, 40), ((2, 3, 5), 1, 1),
+                                      ((2, 3, 5), 2, 3), ((2, 5, 7), 1, 39),
+                                      ((2, 5, 7), 1, 41), ((2, 3, 5), 1, 48)])
 def test_qk_norm_rope(grid, B, H):
     L = grid[0] * grid[1] * grid[2]
     q = inputs.randn_bf16((B, L, H, 128), 21, 2.0)
@@ -58,19 +61,27 @@ def test_qk_norm_rope(grid, B, H):
                     1e-5 * (1 + np.abs(want)).max(axis=-1, keepdims=True))
 
 
-def test_qk_norm_rope_q_only():
-    grid, B, H = (2, 3, 5), 1, 4
+@pytest.mark.parametrize("H", [4, 44])
+@pytest.mark.parametrize("which", ["q", "k"])
+def test_qk_norm_rope_one_tensor(H, which):
+    grid, B = (2, 3, 5), 1
     L = 30
     q = inputs.randn_bf16((B, L, H, 128), 31)
     k = inputs.randn_bf16((B, L, H, 128), 32)
-    wq = inputs.randn_f32((H * 128,), 33)
+    w = inputs.randn_f32((H * 128,), 33)
     g = wan.grid(*grid)
     qg, kg = cuda(q), cuda(k)
-    wan.qk_norm_rope(qg, None, cuda(wq), None, g, wan.rope3d_table(g))
+    if which == "q":
+        wan.qk_norm_rope(qg, None, cuda(w), None, g, wan.rope3d_table(g))
+        done, untouched, x, x_other = qg, kg, q, k
+    else:
+        wan.qk_norm_rope(None, kg, None, cuda(w), g, wan.rope3d_table(g))
+        done, untouched, x, x_other = kg, qg, k, q
     torch.cuda.synchronize()
-    assert torch.equal(kg.cpu(), k)
-    want = oblock.qk_norm_rope(q.double().numpy(), wq.numpy(), grid)
-    _bf16_bound(qg.double().cpu().numpy(), want, 1e-5 * (1 + np.abs(want)))
+    assert torch.equal(untouched.cpu(), x_other)
+    want = oblock.qk_norm_rope(x.double().numpy(), w.numpy(), grid)
+    _bf16_bound(done.double().cpu().numpy(), want,
+                1e-5 * (1 + np.abs(want)).max(axis=-1, keepdims=True))
 
 
 @pytest.mark.parametrize("B,L,D", [(1, 9, 1536), (2, 65, 5120)])

@@ -184,6 +184,82 @@ __global__ void __launch_bounds__(kNrThreads) qk_norm_rope_kernel(
   }
 }
 
+// Register-resident variant for heads <= 2 * kNrMaxRows (all Wan sizes: 12,
+// 24 and 40 heads).  One warp per (token, tensor) item: lane l holds chunk
+// l & 15 of heads l >> 4, l >> 4 + 2, ... in registers, so the row is read
+// from HBM once, in one batch of independent loads, and written once.
+constexpr int kNrMaxRows = 20;
+constexpr int kNrRegThreads = 128;  // 3 CTAs of 168-register threads per SM
+constexpr int kNrRegWarps = kNrRegThreads / 32;
+
+__global__ void __launch_bounds__(kNrRegThreads, 3) qk_norm_rope_reg_kernel(
+    NormRopeArgs a) {
+  const int lane = threadIdx.x & 31;
+  const int c = lane & 15;
+  const int hsub = lane >> 4;
+  const int64_t wstride = static_cast<int64_t>(gridDim.x) * kNrRegWarps;
+  const int hw = a.H * a.W;
+  const float inv_dim = 1.0f / (128.0f * a.heads);
+  // items: (token, tensor) with the present tensors interleaved per token
+  const int ntens = (a.t[0] != nullptr) + (a.t[1] != nullptr);
+  const int first = a.t[0] != nullptr ? 0 : 1;
+  const int64_t items = a.tokens * ntens;
+  for (int64_t it = static_cast<int64_t>(blockIdx.x) * kNrRegWarps +
+                    (threadIdx.x >> 5);
+       it < items; it += wstride) {
+    const int64_t tok = ntens == 2 ? (it >> 1) : it;
+    const int which = ntens == 2 ? static_cast<int>(it & 1) : first;
+    // select, not index: a runtime index into the parameter arrays would
+    // copy them to the stack
+    uint4* t = which ? a.t[1] : a.t[0];
+    const int64_t row0 = tok * a.heads;
+    uint4 r[kNrMaxRows];
+#pragma unroll
+    for (int k = 0; k < kNrMaxRows; ++k) {
+      const int hh = hsub + 2 * k;
+      if (hh < a.heads) r[k] = t[(row0 + hh) * 16 + c];
+    }
+    const int n = static_cast<int>(tok % a.L);
+    const int f = n / hw;
+    const int h = (n / a.W) % a.H;
+    const int w = n % a.W;
+    const float4* tt = a.table + static_cast<int64_t>(f) * 11;
+    const float4* th = a.table + static_cast<int64_t>(a.F + h) * 11;
+    const float4* tw = a.table + static_cast<int64_t>(a.F + a.H + w) * 11;
+    const float4 cs0 = pair_cs(4 * c, tt, th, tw);
+    const float4 cs1 = pair_cs(4 * c + 2, tt, th, tw);
+    float ss = 0.f;
+#pragma unroll
+    for (int k = 0; k < kNrMaxRows; ++k) {
+      if (hsub + 2 * k < a.heads) {
+        const uint32_t vv[4] = {r[k].x, r[k].y, r[k].z, r[k].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 x = bf16x2_to_float2(vv[e]);
+          ss = fmaf(x.x, x.x, fmaf(x.y, x.y, ss));
+        }
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const float fac = rsqrtf(ss * inv_dim + a.eps);
+    const float4* wt = which ? a.w[1] : a.w[0];
+#pragma unroll
+    for (int k = 0; k < kNrMaxRows; ++k) {
+      const int hh = hsub + 2 * k;
+      if (hh < a.heads) {
+        const float4 w0 = __ldg(wt + hh * 32 + 2 * c);
+        const float4 w1 = __ldg(wt + hh * 32 + 2 * c + 1);
+        t[(row0 + hh) * 16 + c] =
+            make_uint4(norm_rot2(r[k].x, fac, w0.x, w0.y, cs0.x, cs0.y),
+                       norm_rot2(r[k].y, fac, w0.z, w0.w, cs0.z, cs0.w),
+                       norm_rot2(r[k].z, fac, w1.x, w1.y, cs1.x, cs1.y),
+                       norm_rot2(r[k].w, fac, w1.z, w1.w, cs1.z, cs1.w));
+      }
+    }
+  }
+}
+
 // ---------------------------------------------------- gated residual ----
 
 constexpr int kResThreads = 256;
@@ -279,11 +355,20 @@ int wan_qk_norm_rope(void* q, void* k, const float* wq, const float* wk,
   a.H = g.H;
   a.W = g.W;
   a.eps = eps;
-  int64_t blocks = (a.tokens + wan::kNrWarps - 1) / wan::kNrWarps;
+  const bool reg = heads <= 2 * wan::kNrMaxRows;
+  const int64_t items = reg ? a.tokens * ((q != nullptr) + (k != nullptr))
+                            : a.tokens;
+  const int wpb = reg ? wan::kNrRegWarps : wan::kNrWarps;
+  int64_t blocks = (items + wpb - 1) / wpb;
   const int64_t cap = static_cast<int64_t>(wan::sm_count_of(dev)) * 8;
   if (cap > 0 && blocks > cap) blocks = cap;
-  wan::qk_norm_rope_kernel<<<static_cast<unsigned>(blocks), wan::kNrThreads,
-                             0, wan::as_stream(s)>>>(a);
+  if (reg)
+    wan::qk_norm_rope_reg_kernel<<<static_cast<unsigned>(blocks),
+                                   wan::kNrRegThreads, 0,
+                                   wan::as_stream(s)>>>(a);
+  else
+    wan::qk_norm_rope_kernel<<<static_cast<unsigned>(blocks),
+                               wan::kNrThreads, 0, wan::as_stream(s)>>>(a);
   return cudaGetLastError() == cudaSuccess ? WAN_OK : WAN_ECUDA;
 }
 
