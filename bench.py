@@ -315,6 +315,19 @@ def hbm_rooflines(dev, g, L, H, n_lat, peak_gbs, n=1 << 28, reps=20):
                            "achieved_gbs": nbytes / (ms / 1e3) / 1e9,
                            "peak_gbs": peak_gbs,
                            "frac": nbytes / (ms / 1e3) / 1e9 / peak_gbs}
+    # Ulysses layout move before the exchange on 8 ranks: Q's 40 heads split
+    # into 8 groups of 5 (rows of 5 x 256 B), every byte read and written once
+    P = 8
+    if H % P == 0:
+        send = torch.empty_like(q)
+        rb = (H // P) * 128 * 2
+        ms = timed(lambda: wan.transpose_blocks(q, send, L, P, rb))
+        nb = 2 * q.numel() * 2
+        out["ulysses_pack_8"] = {"bytes_per_call": nb, "ms": ms,
+                                 "achieved_gbs": nb / (ms / 1e3) / 1e9,
+                                 "peak_gbs": peak_gbs,
+                                 "frac": nb / (ms / 1e3) / 1e9 / peak_gbs}
+        del send
     del q, k
     # AdaLN modulate and gated residual on the fp32 residual stream
     D = H * 128

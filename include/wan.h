@@ -234,6 +234,21 @@ int wan_unipc_step(float* x, float* x_corr, const float* m_prev1,
                    const float* v_uncond, float guide, int64_t n,
                    const double* sigmas, int n_steps, int i, void* s);
 
+/* ------------------------------------------------------------ Ulysses ---
+ * Wan2.2 source reading, ch. 8 "Ulysses": the multi-GPU split trades each
+ * rank's sequence shard of all heads for the whole sequence of its share of
+ * the heads (one all-to-all that scatters one dimension and gathers
+ * another), runs attention, and trades back.
+ *
+ * wan_transpose_blocks: device.  out[j][i][:] = in[i][j][:] for i < a,
+ *   j < b, each row row_bytes long: the outer-dimension swap that makes a
+ *   rank's outgoing chunks (and incoming shards) contiguous around the
+ *   all-to-all.  row_bytes a multiple of 16, in / out 16-byte aligned
+ *   (WAN_EALIGN) and not overlapping (WAN_EINVAL).  Empty sizes do nothing.
+ *   The exchange itself is NCCL's all-to-all.                              */
+int wan_transpose_blocks(const void* in, void* out, int64_t a, int64_t b,
+                         int64_t row_bytes, void* s);
+
 /* ------------------------------------------------------------- status ---
  * Reads (and, if clear != 0, resets) the device status word of the current
  * device: 0 or WAN_ETIMEOUT.  Synchronous (waits for the device).          */

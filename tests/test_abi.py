@@ -162,3 +162,12 @@ def test_argument_checks_without_device(lib):
         == wan.WAN_EINVAL  # q aliases k
     assert L.wan_gated_residual(p, p, p, 1, 4, 6, None) == wan.WAN_EINVAL
     assert L.wan_gated_residual(odd, p, p, 1, 4, 8, None) == wan.WAN_EALIGN
+    big_o = ctypes.c_void_p(1 << 20)
+    assert L.wan_transpose_blocks(p, big_o, 2, 3, 24, None) == wan.WAN_EINVAL
+    assert L.wan_transpose_blocks(p, ctypes.c_void_p(4096 + 64), 2, 3, 16,
+                                  None) == wan.WAN_EINVAL  # overlap
+    assert L.wan_transpose_blocks(odd, big_o, 2, 3, 16, None) \
+        == wan.WAN_EALIGN
+    assert L.wan_transpose_blocks(None, None, 0, 3, 16, None) == wan.WAN_OK
+    assert L.wan_transpose_blocks(None, big_o, 2, 3, 16, None) \
+        == wan.WAN_EINVAL

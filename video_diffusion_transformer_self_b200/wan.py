@@ -83,6 +83,8 @@ _SIGNATURES = {
     "wan_unipc_coeffs": (_I, [_D, _I, _I, ctypes.POINTER(UniPCCoef)]),
     "wan_unipc_step": (_I, [_P, _P, _P, _P, _P, _P, _P, ctypes.c_float,
                             ctypes.c_int64, _D, _I, _I, _P]),
+    "wan_transpose_blocks": (_I, [_P, _P, ctypes.c_int64, ctypes.c_int64,
+                                  ctypes.c_int64, _P]),
     "wan_device_status": (_I, [_I]),
 }
 
@@ -312,6 +314,18 @@ def unipc_step(x, x_corr, m_prev1, m_prev2, m_out, v_cond, v_uncond, guide,
                                 _ptr(m_prev2), _ptr(m_out), _ptr(v_cond),
                                 _ptr(v_uncond), guide, x.numel(), arr, n,
                                 int(i), _stream(stream)), "wan_unipc_step")
+
+
+def transpose_blocks(inp, out, a, b, row_bytes, stream=None):
+    """out[j][i][:] = inp[i][j][:] (i < a, j < b, rows of row_bytes)."""
+    for name, t in (("inp", inp), ("out", out)):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("%s must be a contiguous CUDA tensor" % name)
+        if t.numel() * t.element_size() < a * b * row_bytes:
+            raise ValueError("%s is smaller than a * b * row_bytes" % name)
+    _check(lib().wan_transpose_blocks(_ptr(inp), _ptr(out), int(a), int(b),
+                                      int(row_bytes), _stream(stream)),
+           "wan_transpose_blocks")
 
 
 def device_status(clear=True):
