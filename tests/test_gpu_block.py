@@ -38,11 +38,15 @@ def test_adaln_modulate(B, L, D):
     _bf16_bound(out.double().cpu().numpy(), want, 1e-5 * (1 + np.abs(want)))
 
 
-# heads <= 40 take the register-resident kernel, more heads the two-pass one
+# heads <= 40 take the register-resident kernel (4, 8, 12 or 20 rows per
+# lane by head count), more heads the two-pass one
 @pytest.mark.parametrize("grid,B,H", [((2, 4, 4), 1, 2), ((3, 7, 13), 2, 12),
                                       ((5, 30, 52), 1, 40), ((2, 3, 5), 1, 1),
                                       ((2, 3, 5), 2, 3), ((2, 5, 7), 1, 39),
-                                      ((2, 5, 7), 1, 41), ((2, 3, 5), 1, 48)])
+                                      ((2, 5, 7), 1, 41), ((2, 3, 5), 1, 48),
+                                      ((2, 3, 5), 1, 8), ((2, 3, 5), 1, 9),
+                                      ((2, 3, 5), 1, 16), ((2, 3, 5), 2, 24),
+                                      ((2, 3, 5), 1, 25)])
 def test_qk_norm_rope(grid, B, H):
     L = grid[0] * grid[1] * grid[2]
     q = inputs.randn_bf16((B, L, H, 128), 21, 2.0)

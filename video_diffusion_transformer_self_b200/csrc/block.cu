@@ -184,16 +184,24 @@ __global__ void __launch_bounds__(kNrThreads) qk_norm_rope_kernel(
   }
 }
 
-// Register-resident variant for heads <= 2 * kNrMaxRows (all Wan sizes: 12,
-// 24 and 40 heads).  One warp per (token, tensor) item: lane l holds chunk
+// Register-resident variant for heads <= 2 * kRows (all Wan sizes: 12, 24
+// and 40 heads).  One warp per (token, tensor) item: lane l holds chunk
 // l & 15 of heads l >> 4, l >> 4 + 2, ... in registers, so the row is read
-// from HBM once, in one batch of independent loads, and written once.
+// from HBM once, in one batch of independent loads, and written once.  kRows
+// is picked from the head count so that small rows keep a high occupancy.
 constexpr int kNrMaxRows = 20;
-constexpr int kNrRegThreads = 128;  // 3 CTAs of 168-register threads per SM
+constexpr int kNrRegThreads = 128;
 constexpr int kNrRegWarps = kNrRegThreads / 32;
 
-__global__ void __launch_bounds__(kNrRegThreads, 3) qk_norm_rope_reg_kernel(
-    NormRopeArgs a) {
+// resident CTAs per SM that each row-register budget allows
+template <int kRows>
+constexpr int nr_min_blocks() {
+  return kRows <= 4 ? 8 : kRows <= 12 ? 6 : 3;
+}
+
+template <int kRows>
+__global__ void __launch_bounds__(kNrRegThreads, nr_min_blocks<kRows>())
+    qk_norm_rope_reg_kernel(NormRopeArgs a) {
   const int lane = threadIdx.x & 31;
   const int c = lane & 15;
   const int hsub = lane >> 4;
@@ -213,9 +221,9 @@ __global__ void __launch_bounds__(kNrRegThreads, 3) qk_norm_rope_reg_kernel(
     // copy them to the stack
     uint4* t = which ? a.t[1] : a.t[0];
     const int64_t row0 = tok * a.heads;
-    uint4 r[kNrMaxRows];
+    uint4 r[kRows];
 #pragma unroll
-    for (int k = 0; k < kNrMaxRows; ++k) {
+    for (int k = 0; k < kRows; ++k) {
       const int hh = hsub + 2 * k;
       if (hh < a.heads) r[k] = t[(row0 + hh) * 16 + c];
     }
@@ -230,7 +238,7 @@ __global__ void __launch_bounds__(kNrRegThreads, 3) qk_norm_rope_reg_kernel(
     const float4 cs1 = pair_cs(4 * c + 2, tt, th, tw);
     float ss = 0.f;
 #pragma unroll
-    for (int k = 0; k < kNrMaxRows; ++k) {
+    for (int k = 0; k < kRows; ++k) {
       if (hsub + 2 * k < a.heads) {
         const uint32_t vv[4] = {r[k].x, r[k].y, r[k].z, r[k].w};
 #pragma unroll
@@ -245,7 +253,7 @@ __global__ void __launch_bounds__(kNrRegThreads, 3) qk_norm_rope_reg_kernel(
     const float fac = rsqrtf(ss * inv_dim + a.eps);
     const float4* wt = which ? a.w[1] : a.w[0];
 #pragma unroll
-    for (int k = 0; k < kNrMaxRows; ++k) {
+    for (int k = 0; k < kRows; ++k) {
       const int hh = hsub + 2 * k;
       if (hh < a.heads) {
         const float4 w0 = __ldg(wt + hh * 32 + 2 * c);
@@ -362,10 +370,17 @@ int wan_qk_norm_rope(void* q, void* k, const float* wq, const float* wk,
   int64_t blocks = (items + wpb - 1) / wpb;
   const int64_t cap = static_cast<int64_t>(wan::sm_count_of(dev)) * 8;
   if (cap > 0 && blocks > cap) blocks = cap;
-  if (reg)
-    wan::qk_norm_rope_reg_kernel<<<static_cast<unsigned>(blocks),
-                                   wan::kNrRegThreads, 0,
-                                   wan::as_stream(s)>>>(a);
+  const unsigned nb = static_cast<unsigned>(blocks);
+  cudaStream_t st_ = wan::as_stream(s);
+  if (reg && heads <= 8)
+    wan::qk_norm_rope_reg_kernel<4><<<nb, wan::kNrRegThreads, 0, st_>>>(a);
+  else if (reg && heads <= 16)
+    wan::qk_norm_rope_reg_kernel<8><<<nb, wan::kNrRegThreads, 0, st_>>>(a);
+  else if (reg && heads <= 24)
+    wan::qk_norm_rope_reg_kernel<12><<<nb, wan::kNrRegThreads, 0, st_>>>(a);
+  else if (reg)
+    wan::qk_norm_rope_reg_kernel<wan::kNrMaxRows>
+        <<<nb, wan::kNrRegThreads, 0, st_>>>(a);
   else
     wan::qk_norm_rope_kernel<<<static_cast<unsigned>(blocks),
                                wan::kNrThreads, 0, wan::as_stream(s)>>>(a);
