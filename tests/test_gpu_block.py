@@ -25,8 +25,10 @@ def _bf16_bound(got, want, extra):
     assert np.all(err <= bound), float(np.max(err / bound))
 
 
+# row lengths across the 3, 6, 10 and 16 float4-per-thread variants
 @pytest.mark.parametrize("B,L,D", [(1, 7, 1536), (2, 33, 5120), (1, 5, 8),
-                                   (3, 4, 8192)])
+                                   (3, 4, 8192), (1, 5, 3072), (2, 3, 6144),
+                                   (1, 3, 1540), (1, 2, 5124)])
 def test_adaln_modulate(B, L, D):
     x = inputs.randn_f32((B, L, D), 11, 3.0) + 0.5
     shift = inputs.randn_f32((B, D), 12, 0.2)

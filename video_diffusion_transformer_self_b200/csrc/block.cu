@@ -38,6 +38,9 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
   return t;
 }
 
+// kVec float4 per thread (D <= 128 * 4 * kVec), picked from D so that the
+// row's registers, and so the occupancy, follow the row length.
+template <int kVec>
 __global__ void __launch_bounds__(kModThreads)
     adaln_modulate_kernel(const float4* __restrict__ x,
                           const float4* __restrict__ shift,
@@ -47,10 +50,10 @@ __global__ void __launch_bounds__(kModThreads)
   const int64_t tok = blockIdx.x;          // b * L + l
   const int b = static_cast<int>(tok / L);
   const float4* xr = x + tok * D4;
-  float4 v[kModMaxVec];
+  float4 v[kVec];
   float s = 0.f;
 #pragma unroll
-  for (int u = 0; u < kModMaxVec; ++u) {
+  for (int u = 0; u < kVec; ++u) {
     const int i = threadIdx.x + u * kModThreads;
     if (i < D4) {
       v[u] = xr[i];
@@ -61,7 +64,7 @@ __global__ void __launch_bounds__(kModThreads)
   const float mean = block_sum(s, red) * inv_d;
   float ss = 0.f;
 #pragma unroll
-  for (int u = 0; u < kModMaxVec; ++u) {
+  for (int u = 0; u < kVec; ++u) {
     const int i = threadIdx.x + u * kModThreads;
     if (i < D4) {
       const float a = v[u].x - mean, bb = v[u].y - mean;
@@ -72,7 +75,7 @@ __global__ void __launch_bounds__(kModThreads)
   const float rstd = rsqrtf(block_sum(ss, red) * inv_d + eps);
   uint2* orow = out + tok * D4;
 #pragma unroll
-  for (int u = 0; u < kModMaxVec; ++u) {
+  for (int u = 0; u < kVec; ++u) {
     const int i = threadIdx.x + u * kModThreads;
     if (i < D4) {
       const float4 sh = __ldg(shift + static_cast<int64_t>(b) * D4 + i);
@@ -325,12 +328,26 @@ int wan_adaln_modulate(const float* x, const float* shift, const float* scale,
     return WAN_EALIGN;
   int st = wan::check_device(nullptr);
   if (st != WAN_OK) return st;
-  wan::adaln_modulate_kernel<<<static_cast<unsigned>(B * L),
-                               wan::kModThreads, 0, wan::as_stream(s)>>>(
-      reinterpret_cast<const float4*>(x),
-      reinterpret_cast<const float4*>(shift),
-      reinterpret_cast<const float4*>(scale), static_cast<uint2*>(out), L,
-      D / 4, eps);
+  const int D4 = D / 4;
+  const int vec = (D4 + wan::kModThreads - 1) / wan::kModThreads;
+  const unsigned nb = static_cast<unsigned>(B * L);
+  cudaStream_t st_ = wan::as_stream(s);
+  const float4* x4 = reinterpret_cast<const float4*>(x);
+  const float4* sh4 = reinterpret_cast<const float4*>(shift);
+  const float4* sc4 = reinterpret_cast<const float4*>(scale);
+  uint2* o2 = static_cast<uint2*>(out);
+  if (vec <= 3)
+    wan::adaln_modulate_kernel<3><<<nb, wan::kModThreads, 0, st_>>>(
+        x4, sh4, sc4, o2, L, D4, eps);
+  else if (vec <= 6)
+    wan::adaln_modulate_kernel<6><<<nb, wan::kModThreads, 0, st_>>>(
+        x4, sh4, sc4, o2, L, D4, eps);
+  else if (vec <= 10)
+    wan::adaln_modulate_kernel<10><<<nb, wan::kModThreads, 0, st_>>>(
+        x4, sh4, sc4, o2, L, D4, eps);
+  else
+    wan::adaln_modulate_kernel<wan::kModMaxVec>
+        <<<nb, wan::kModThreads, 0, st_>>>(x4, sh4, sc4, o2, L, D4, eps);
   return cudaGetLastError() == cudaSuccess ? WAN_OK : WAN_ECUDA;
 }
 
