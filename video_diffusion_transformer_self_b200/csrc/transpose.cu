@@ -22,7 +22,7 @@ constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 
 // One warp per output row (j, i): one division per row, lanes copy
-// consecutive 16-byte chunks.
+// consecutive 16-byte chunks, four loads in flight per lane.
 __global__ void __launch_bounds__(kThreads)
     transpose_blocks_kernel(const uint4* __restrict__ in,
                             uint4* __restrict__ out, int64_t a, int64_t b,
@@ -37,7 +37,16 @@ __global__ void __launch_bounds__(kThreads)
     const int64_t i = r - j * a;
     const uint4* src = in + (i * b + j) * row16;
     uint4* dst = out + r * row16;
-    for (int64_t c = lane; c < row16; c += 32) dst[c] = src[c];
+    // up to four loads in flight per lane before the stores
+    for (int64_t c0 = lane; c0 < row16; c0 += 4 * 32) {
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (c0 + u * 32 < row16) v[u] = src[c0 + u * 32];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (c0 + u * 32 < row16) dst[c0 + u * 32] = v[u];
+    }
   }
 }
 
