@@ -575,10 +575,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       float s[BN];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(s_col + c * 32, s + c * 32);
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld_wait32(s + c * 32);
+      static_assert(BN == 128, "one 128-column TMEM load per score row");
+      tmem_ld128(s_col, s);
+      tmem_ld_wait128(s);
       const int lim = row_lim - j * BN;  // valid keys of this row here
       // warp-uniform: any masked row sends the warp down the exact path
       const bool masked = __any_sync(0xffffffffu, lim < BN);
