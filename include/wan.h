@@ -249,6 +249,18 @@ int wan_unipc_step(float* x, float* x_corr, const float* m_prev1,
 int wan_transpose_blocks(const void* in, void* out, int64_t a, int64_t b,
                          int64_t row_bytes, void* s);
 
+/* ---------------------------------------------------- wait self-test ---
+ * wan_wait_selftest: launches one warp on stream s that waits, with the
+ * library's bounded mbarrier wait, on a barrier needing one arrival and
+ * given `arrive` (0 or 1) of them.  With 0 the wait runs out after its 2 s
+ * limit, WAN_ETIMEOUT is recorded in the device status word
+ * (wan_device_status) and the kernel returns, leaving the context usable;
+ * with 1 it completes at once.  It lets a test check the timeout path
+ * without a fault or a hang.  The pages have no counterpart: this is a
+ * check of the library's own failure handling.  WAN_EINVAL for other
+ * values of arrive.                                                        */
+int wan_wait_selftest(int arrive, void* s);
+
 /* ------------------------------------------------------------- status ---
  * Reads (and, if clear != 0, resets) the device status word of the current
  * device: 0 or WAN_ETIMEOUT.  Synchronous (waits for the device).          */

@@ -679,6 +679,26 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// One warp waits, with the same bounded wait the attention kernel uses, on
+// an mbarrier that needs one arrival and receives `arrive` (0 or 1).  With
+// none the wait runs out after kWaitLimitNs, records WAN_ETIMEOUT in the
+// device status word and the kernel returns: the timeout path can be
+// checked without a fault or a hang.
+__global__ void __launch_bounds__(32) wait_selftest_kernel(int arrive) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int s_abort;
+  if (threadIdx.x == 0) {
+    s_abort = 0;
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  if (arrive && threadIdx.x == 0) mbar_arrive(&bar);
+  __syncwarp();
+  volatile int* abort_flag = &s_abort;
+  wait_warp(&bar, 0, abort_flag, &g_wan_status);
+}
+
 // ------------------------------------------------------------------ host --
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType,
@@ -879,6 +899,14 @@ int wan_cross_attn(const void* q, const void* k_ctx, const void* v_ctx,
   a.q_offset = 0;
   for (int i = 0; i < B; ++i) a.lens[i] = ctx_lens[i];
   return launch<0>(mq, mk, mv, a, B, as_stream(s));
+}
+
+int wan_wait_selftest(int arrive, void* s) {
+  if (arrive != 0 && arrive != 1) return WAN_EINVAL;
+  int st = wan::check_device(nullptr);
+  if (st != WAN_OK) return st;
+  wan::wait_selftest_kernel<<<1, 32, 0, wan::as_stream(s)>>>(arrive);
+  return cudaGetLastError() == cudaSuccess ? WAN_OK : WAN_ECUDA;
 }
 
 int wan_device_status(int clear) {

@@ -85,6 +85,7 @@ _SIGNATURES = {
                             ctypes.c_int64, _D, _I, _I, _P]),
     "wan_transpose_blocks": (_I, [_P, _P, ctypes.c_int64, ctypes.c_int64,
                                   ctypes.c_int64, _P]),
+    "wan_wait_selftest": (_I, [_I, _P]),
     "wan_device_status": (_I, [_I]),
 }
 
@@ -326,6 +327,12 @@ def transpose_blocks(inp, out, a, b, row_bytes, stream=None):
     _check(lib().wan_transpose_blocks(_ptr(inp), _ptr(out), int(a), int(b),
                                       int(row_bytes), _stream(stream)),
            "wan_transpose_blocks")
+
+
+def wait_selftest(arrive, stream=None):
+    """Launch the bounded-wait self-test kernel (see include/wan.h)."""
+    _check(lib().wan_wait_selftest(int(arrive), _stream(stream)),
+           "wan_wait_selftest")
 
 
 def device_status(clear=True):
