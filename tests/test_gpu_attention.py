@@ -60,6 +60,7 @@ SELF_CASES = [
     ((2, 8, 16), 1, 2),     # exactly 2 tiles
     ((1, 1, 1), 1, 2),      # single token
     ((1, 3, 43), 1, 1),     # 129 tokens: one full tile + 1
+    ((1, 1, 127), 1, 2),    # 127 tokens: one tile short of a row
     ((2, 12, 16), 1, 1),    # 384 tokens: 3 tiles, second CTA half empty
     ((1, 5, 77), 2, 1),     # 385 tokens: 4 tiles, last holds 1 row
 ]
