@@ -421,6 +421,26 @@ def causal_rooflines(dev, peak_tflops, reps=5):
     return out
 
 
+def cross_roofline(B, L, H, Lk, lens, ms, peak_tflops, peak_gbs):
+    """Cross-attention launch of the timed step (CUDA events around it).
+    FLOPs count the true text lengths, 4 * L * len_b * 128 * H per batch row
+    (and, for reference, the padded Lk); bytes are Q read and O written
+    (B * L * H * 256 each) plus the len_b valid K and V rows.  Its
+    arithmetic intensity (about len_b FLOP per byte) is near the B200 ridge,
+    so both fractions are given."""
+    fl = sum(4.0 * L * n * 128 * H for n in lens)
+    fl_pad = 4.0 * B * L * Lk * 128 * H
+    nb = 2.0 * B * L * H * 256 + sum(2.0 * n * H * 256 for n in lens)
+    tf = fl / (ms / 1e3) / 1e12
+    gbs = nb / (ms / 1e3) / 1e9
+    return {"kernel": "attn_fwd_kernel cross-attention", "ms": ms,
+            "text_lens": list(lens), "flops": fl, "bytes": nb,
+            "tflops": tf, "tflops_padded_lk": fl_pad / (ms / 1e3) / 1e12,
+            "frac_of_sustained_tensor_peak": tf / peak_tflops,
+            "gbs": gbs, "frac_of_hbm_peak": gbs / peak_gbs,
+            "intensity_flop_per_byte": fl / nb}
+
+
 def run_wan(args, w, rank, world, local_rank):
     import numpy as np
     import torch
@@ -463,6 +483,7 @@ def run_wan(args, w, rank, world, local_rank):
     flops_self = 4.0 * B * H * L * L * 128
 
     ev_pairs = []
+    ev_cross = []
 
     def step(i, timed):
         s0, s1 = sigmas[i % w.steps], sigmas[i % w.steps + 1]
@@ -480,6 +501,10 @@ def run_wan(args, w, rank, world, local_rank):
             e1.record(stream)
             ev_pairs.append((e0, e1))
         wan.cross_attn(o, d["k_ctx"], d["v_ctx"], oc, lens)
+        if timed:
+            e2 = torch.cuda.Event(enable_timing=True)
+            e2.record(stream)
+            ev_cross.append((e1, e2))
         wan.fm_step(d["x"], d["v_cond"], d["v_uncond"], guide, s0, s1)
 
     launches_per_step = 4 if args.rope == "pre" else 3
@@ -517,7 +542,10 @@ def run_wan(args, w, rank, world, local_rank):
     # self-attention launch time (the RoPE pass of --rope pre excluded)
     attn_ms = [a.elapsed_time(b) for a, b in ev_pairs]
     attn_avg = sum(attn_ms) / len(attn_ms)
-    ms, attn_avg = max_over_ranks([ms, attn_avg], dist, dev)
+    cross_ms = [a.elapsed_time(b) for a, b in ev_cross]
+    cross_avg = sum(cross_ms) / len(cross_ms)
+    ms, attn_avg, cross_avg = max_over_ranks([ms, attn_avg, cross_avg], dist,
+                                             dev)
 
     # ----- end to end: host buffers in, results out, every step -----
     # Each step copies its inputs from pinned host memory and reads back its
@@ -644,6 +672,8 @@ def run_wan(args, w, rank, world, local_rank):
                                    "long step)",
             "avg_launch_ms": attn_avg,
         },
+        "cross_attn": cross_roofline(B, L, H, w.text_tokens, lens, cross_avg,
+                                     peak, float(pk.get("hbm_gbs", 6650.0))),
         "gpu_launches": launches_per_step * args.steps,
         "e2e": e2e,
         "clocks": clk,
