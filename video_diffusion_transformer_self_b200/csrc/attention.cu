@@ -9,18 +9,21 @@
 // prompt's true length take no part.  Wan paper explainer, section "Text
 // encoder": softmax(Q K_text^T / sqrt(d_k)) V_text.
 //
-// One CTA per (256 query rows = two 128-row tiles, head, batch row).  The two
-// tiles ping-pong: while the softmax of one tile runs, the tensor cores run
-// the other tile's P V and next Q K^T, so neither waits on the other.
+// Work items are (256 query rows = two 128-row tiles, head, batch row); a CTA
+// runs one item, or, for cross-attention, walks items persistently (one CTA
+// per SM) so that the next item's Q loads while the current one drains.  The
+// two tiles ping-pong: while the softmax of one tile runs, the tensor cores
+// run the other tile's P V and next Q K^T, so neither waits on the other.
 // Warp roles (384 threads, registers rebalanced with setmaxnreg):
 //   warps 0-3 / 4-7  softmax of tile 0 / tile 1: thread r owns query row r
 //              (TMEM lane r).  Reads the 128x128 fp32 score tile from TMEM,
 //              keeps the running row max (log2 units) and sum, rescales O
 //              in TMEM when the max grows by more than 2^8 (exact after the
 //              final O / l), writes P (bf16) back into TMEM over its
-//              scores, and writes the bf16 epilogue.  A quarter of the exponentials
-//              run on the FMA pipe (exp2_fma2) to offload the MUFU unit.
-//   warp 8     TMA producer: the two Q tiles once, then K (3-stage ring) and
+//              scores, and writes the bf16 epilogue.  A quarter of the
+//              exponentials run on the FMA pipe (exp2_fma2) to offload the
+//              MUFU unit.
+//   warp 8     TMA producer: each item's two Q tiles, then K (3-stage ring) and
 //              V (2-stage ring).
 //   warp 9     MMA issuer (one lane): S_t = Q_t K^T (both operands K-major in
 //              smem) and O_t += P_t V (P from TMEM, V MN-major in smem), in
@@ -87,8 +90,37 @@ struct AttnArgs {
   int cross;            // 1: per-batch key length from lens[]
   int chunk;            // > 0: block-causal, chunk length in tokens
   int q_offset;         // block-causal: absolute position of query row 0
+  int n_tiles_x;        // 256-row query tile pairs per (head, batch row)
+  int items;            // n_tiles_x * heads * B work items
   int lens[MAX_CROSS_BATCH];
 };
+
+// One work item: a pair of 128-row query tiles of one (head, batch row).
+// Items are numbered tile-fastest, then head, then batch row, the order a
+// (tiles, heads, B) grid launches in; block-causal items run heaviest first
+// within a head.
+struct Item {
+  int q0, head, b, kv_len, nblk;
+};
+
+__device__ __forceinline__ Item item_of(const AttnArgs& a, int it) {
+  Item c;
+  const int tx = it % a.n_tiles_x;
+  const int rest = it / a.n_tiles_x;
+  c.head = rest % a.heads;
+  c.b = rest / a.heads;
+  const int tile_x = a.chunk ? (a.n_tiles_x - 1 - tx) : tx;
+  c.q0 = tile_x * (QT * BM);
+  int kv = a.cross ? a.lens[c.b] : a.Lk;
+  if (a.chunk) {
+    // keys visible to the last query row of this item
+    const int last = min(c.q0 + QT * BM, a.Lq) - 1 + a.q_offset;
+    kv = min(a.Lk, (last / a.chunk + 1) * a.chunk);
+  }
+  c.kv_len = kv;
+  c.nblk = (kv + BN - 1) / BN;
+  return c;
+}
 
 // Barrier slots.
 enum : int {
@@ -101,8 +133,10 @@ enum : int {
   B_VEMPTY = B_VFULL + NSV,
   B_SFULL = B_VEMPTY + NSV,  // per tile
   B_PPART = B_SFULL + QT,    // per tile and part, one arrival per warp
-  B_OFINAL = B_PPART + QT * NPART,  // per tile, last PV only (single phase)
-  B_DRAIN = B_OFINAL + QT,
+  B_OFINAL = B_PPART + QT * NPART,  // per tile: an item's last PV done
+  B_OFREE = B_OFINAL + QT,   // per tile: O of the item read out (4 warps)
+  B_QEMPTY = B_OFREE + QT,   // an item's S MMAs done: Q buffer reusable
+  B_DRAIN = B_QEMPTY + 1,
   NBAR = B_DRAIN + 1
 };
 
@@ -267,8 +301,9 @@ __device__ __forceinline__ void exp_store_chunks(const float* s, float c2,
                                                  float m, uint32_t pcol,
                                                  float2 (&acc)[4], int c0,
                                                  int c1) {
-  // Chunks [c0, c1) of 32 keys (constants after unrolling): p = 2^(s c2 - m), packed to bf16 pairs into
-  // the tile's P columns (16 per chunk), p summed into acc in fp32.
+  // Chunks [c0, c1) of 32 keys (constants after unrolling):
+  // p = 2^(s c2 - m), packed to bf16 pairs into the tile's P columns (16 per
+  // chunk), p summed into acc in fp32.
   const float2 c22 = make_float2(c2, c2);
   const float2 nm2 = make_float2(-m, -m);
 #pragma unroll
@@ -293,7 +328,10 @@ __device__ __forceinline__ void exp_store_chunks(const float* s, float c2,
   }
 }
 
-template <int kRope>
+// kPersist: the CTA walks items it = blockIdx.x, + gridDim.x, ...;
+// otherwise it runs item blockIdx.x only (the loops below then run once and
+// compile to straight-line code).
+template <int kRope, int kPersist>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
@@ -306,18 +344,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // Block-causal CTAs differ in work; the heaviest (last) start first.
-  const int tile_x = args.chunk ? (gridDim.x - 1 - blockIdx.x) : blockIdx.x;
-  const int q0 = tile_x * (QT * BM);
-  const int head = blockIdx.y;
-  const int b = blockIdx.z;
-  int kv_len = args.cross ? args.lens[b] : args.Lk;
-  if (args.chunk) {
-    // keys visible to the last query row of this CTA
-    const int last = min(q0 + QT * BM, args.Lq) - 1 + args.q_offset;
-    kv_len = min(args.Lk, (last / args.chunk + 1) * args.chunk);
-  }
-  const int nblk = (kv_len + BN - 1) / BN;
+  // Every role walks the same items, it = blockIdx.x, + gridDim.x, ...; the
+  // barrier phases of the K / V rings and of S / P run on across items
+  // (g counts key blocks over all of this CTA's items, n counts items).
   volatile int* abort_flag = &s_abort;
   int* status = &g_wan_status;
 
@@ -342,9 +371,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int t = 0; t < QT; ++t) {
       mbar_init(&bar[B_SFULL + t], 1);
-      for (int q = 0; q < NPART; ++q) mbar_init(&bar[B_PPART + t * NPART + q], 4);
+      for (int q = 0; q < NPART; ++q)
+        mbar_init(&bar[B_PPART + t * NPART + q], 4);
       mbar_init(&bar[B_OFINAL + t], 1);
+      mbar_init(&bar[B_OFREE + t], 4);
     }
+    mbar_init(&bar[B_QEMPTY], 1);
     mbar_init(&bar[B_DRAIN], 1);
     fence_mbar_init();
   }
@@ -365,50 +397,65 @@ __global__ void __launch_bounds__(kThreads, 1)
         prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_k);
         prefetch_tmap(&tm_v);
-        mbar_expect_tx(&bar[B_QFULL], QT * TILE);
-        for (int t = 0; t < QT; ++t) {
-          tma_load_4d(sQ + t * TILE, &tm_q, &bar[B_QFULL], 0, head,
-                      q0 + t * BM, b);
-          tma_load_4d(sQ + t * TILE + HALF, &tm_q, &bar[B_QFULL], 64, head,
-                      q0 + t * BM, b);
-        }
       }
       bool ok = true;
-      int nk = 0, nv = 0;  // K / V tiles issued
-      for (int j = 0; j < nblk && ok; ++j) {
-        const int sk = j % NSK, uk = j / NSK;
-        if (uk > 0)
-          ok = wait_warp(&bar[B_KEMPTY + sk], (uk - 1) & 1, abort_flag, status);
+      int nq = 0, nk = 0, nv = 0;  // Q pairs / K / V tiles issued
+      for (int it = blockIdx.x, n = 0;
+           it < (kPersist ? args.items : blockIdx.x + 1) && ok;
+           it += gridDim.x, ++n) {
+        const Item c = item_of(args, it);
+        // the previous item's S MMAs must be done with the Q buffer
+        if (n > 0)
+          ok = wait_warp(&bar[B_QEMPTY], (n - 1) & 1, abort_flag, status);
         if (!ok) break;
         if (leader) {
-          mbar_expect_tx(&bar[B_KFULL + sk], TILE);
-          tma_load_4d(sK + sk * TILE, &tm_k, &bar[B_KFULL + sk], 0, head,
-                      j * BN, b);
-          tma_load_4d(sK + sk * TILE + HALF, &tm_k, &bar[B_KFULL + sk], 64,
-                      head, j * BN, b);
+          mbar_expect_tx(&bar[B_QFULL], QT * TILE);
+          for (int t = 0; t < QT; ++t) {
+            tma_load_4d(sQ + t * TILE, &tm_q, &bar[B_QFULL], 0, c.head,
+                        c.q0 + t * BM, c.b);
+            tma_load_4d(sQ + t * TILE + HALF, &tm_q, &bar[B_QFULL], 64,
+                        c.head, c.q0 + t * BM, c.b);
+          }
         }
-        ++nk;
-        const int sv = j % NSV, uv = j / NSV;
-        if (uv > 0)
-          ok = wait_warp(&bar[B_VEMPTY + sv], (uv - 1) & 1, abort_flag, status);
-        if (!ok) break;
-        if (leader) {
-          mbar_expect_tx(&bar[B_VFULL + sv], TILE);
-          tma_load_4d(sV + sv * TILE, &tm_v, &bar[B_VFULL + sv], 0, head,
-                      j * BN, b);
-          tma_load_4d(sV + sv * TILE + HALF, &tm_v, &bar[B_VFULL + sv], 64,
-                      head, j * BN, b);
+        ++nq;
+        for (int j = 0; j < c.nblk && ok; ++j) {
+          const int g = nk;  // key blocks issued so far == this block's g
+          const int sk = g % NSK, uk = g / NSK;
+          if (uk > 0)
+            ok = wait_warp(&bar[B_KEMPTY + sk], (uk - 1) & 1, abort_flag,
+                           status);
+          if (!ok) break;
+          if (leader) {
+            mbar_expect_tx(&bar[B_KFULL + sk], TILE);
+            tma_load_4d(sK + sk * TILE, &tm_k, &bar[B_KFULL + sk], 0, c.head,
+                        j * BN, c.b);
+            tma_load_4d(sK + sk * TILE + HALF, &tm_k, &bar[B_KFULL + sk], 64,
+                        c.head, j * BN, c.b);
+          }
+          ++nk;
+          const int sv = g % NSV, uv = g / NSV;
+          if (uv > 0)
+            ok = wait_warp(&bar[B_VEMPTY + sv], (uv - 1) & 1, abort_flag,
+                           status);
+          if (!ok) break;
+          if (leader) {
+            mbar_expect_tx(&bar[B_VFULL + sv], TILE);
+            tma_load_4d(sV + sv * TILE, &tm_v, &bar[B_VFULL + sv], 0, c.head,
+                        j * BN, c.b);
+            tma_load_4d(sV + sv * TILE + HALF, &tm_v, &bar[B_VFULL + sv], 64,
+                        c.head, j * BN, c.b);
+          }
+          ++nv;
+          __syncwarp();
         }
-        ++nv;
-        __syncwarp();
       }
       if (*abort_flag) {
         // Let copies already issued land before the CTA leaves.
-        wait_warp_drain(&bar[B_QFULL], 0, status);
-        for (int j = (nk > NSK ? nk - NSK : 0); j < nk; ++j)
-          wait_warp_drain(&bar[B_KFULL + j % NSK], (j / NSK) & 1, status);
-        for (int j = (nv > NSV ? nv - NSV : 0); j < nv; ++j)
-          wait_warp_drain(&bar[B_VFULL + j % NSV], (j / NSV) & 1, status);
+        if (nq > 0) wait_warp_drain(&bar[B_QFULL], (nq - 1) & 1, status);
+        for (int g = (nk > NSK ? nk - NSK : 0); g < nk; ++g)
+          wait_warp_drain(&bar[B_KFULL + g % NSK], (g / NSK) & 1, status);
+        for (int g = (nv > NSV ? nv - NSV : 0); g < nv; ++g)
+          wait_warp_drain(&bar[B_VFULL + g % NSV], (g / NSV) & 1, status);
       }
     } else if (warp == 9) {
       // -------------------------------------------------------- MMA issuer --
@@ -422,9 +469,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool leader = elect_one();
       // S_t(j) = Q_t K(j)^T into the score buffer of tile t.  Descriptor
       // arithmetic runs in all lanes (warp-uniform); one lane issues.
-      auto issue_s = [&](int t, int j) {
+      auto issue_s = [&](int t, int g) {
         const uint64_t a0 = dq + ((t * TILE) >> 4);
-        const uint64_t b0 = dk + (((j % NSK) * TILE) >> 4);
+        const uint64_t b0 = dk + (((g % NSK) * TILE) >> 4);
         const uint32_t d = tmem + t * 128;
         if (leader) {
 #pragma unroll
@@ -438,9 +485,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
       };
-      // O_t += P_t(i) V(i) over the keys of P part `part`.
-      auto issue_pv_part = [&](int t, int i, int part) {
-        const uint64_t b0 = dv + (((i % NSV) * TILE) >> 4);
+      // O_t += P_t V over the keys of P part `part`; g is the block's global
+      // count (ring stage), jl its index within the item (accumulate flag).
+      auto issue_pv_part = [&](int t, int g, int jl, int part) {
+        const uint64_t b0 = dv + (((g % NSV) * TILE) >> 4);
         const uint32_t d = tmem + TM_O + t * 128;
         const uint32_t a = tmem + t * 128;
         if (leader) {
@@ -450,7 +498,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int kk = 0; kk < KPP; ++kk) {
             const int k = part * KPP + kk;
             umma_ts(d, a + k * 8, b0 + ((k * 2048) >> 4), IDESC_PV,
-                    (i > 0 || k > 0) ? 1u : 0u);
+                    (jl > 0 || k > 0) ? 1u : 0u);
           }
         }
         __syncwarp();
@@ -460,15 +508,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (leader) umma_commit(b);
         __syncwarp();
       };
-      // Waits for V(i) and clears its text-padding rows: they may hold
-      // anything (NaN included), and P is 0 there but 0 * NaN is not.
-      auto ready_v = [&](int i) -> bool {
-        if (!wait_warp(&bar[B_VFULL + i % NSV], (i / NSV) & 1, abort_flag,
+      // Waits for V of block g and clears its text-padding rows: they may
+      // hold anything (NaN included), and P is 0 there but 0 * NaN is not.
+      auto ready_v = [&](int g, int jl, int kv_len) -> bool {
+        if (!wait_warp(&bar[B_VFULL + g % NSV], (g / NSV) & 1, abort_flag,
                        status))
           return false;
-        if (args.cross && kv_len < (i + 1) * BN) {
-          const int first = kv_len - i * BN;
-          uint8_t* vt = sV + (i % NSV) * TILE;
+        if (args.cross && kv_len < (jl + 1) * BN) {
+          const int first = kv_len - jl * BN;
+          uint8_t* vt = sV + (g % NSV) * TILE;
           for (int idx = lane; idx < (BN - first) * 16; idx += 32) {
             const int r = first + (idx >> 4);
             const int c = idx & 15;
@@ -480,50 +528,66 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         return true;
       };
-      // O_t += P_t(i) V(i), each part issued as soon as the softmax warps
-      // have published it.
-      auto pv = [&](int t, int i) -> bool {
+      // O_t += P_t V for block g (index jl in item n), each part issued as
+      // soon as the softmax warps have published it.  An item's first P V
+      // overwrites O_t, so it also waits until the previous item's O_t has
+      // been read out.
+      auto pv = [&](int t, int g, int jl, int n) -> bool {
+        if (jl == 0 && n > 0 &&
+            !wait_warp(&bar[B_OFREE + t], (n - 1) & 1, abort_flag, status))
+          return false;
         for (int part = 0; part < NPART; ++part) {
-          if (!wait_warp(&bar[B_PPART + t * NPART + part], i & 1, abort_flag,
+          if (!wait_warp(&bar[B_PPART + t * NPART + part], g & 1, abort_flag,
                          status))
             return false;
           tc_fence_after();
-          issue_pv_part(t, i, part);
+          issue_pv_part(t, g, jl, part);
         }
         return true;
       };
-      bool ok = wait_warp(&bar[kRope ? B_QREADY : B_QFULL], 0, abort_flag,
-                          status);
-      for (int j = 0; j < nblk && ok; ++j) {
-        const int sk = j % NSK;
-        if (j > 0) {
-          ok = ready_v(j - 1) && pv(0, j - 1);
+      bool ok = true;
+      int g0 = 0;  // key blocks of earlier items
+      for (int it = blockIdx.x, n = 0;
+           it < (kPersist ? args.items : blockIdx.x + 1) && ok;
+           it += gridDim.x, ++n) {
+        const Item c = item_of(args, it);
+        ok = wait_warp(&bar[kRope ? B_QREADY : B_QFULL], n & 1, abort_flag,
+                       status);
+        for (int j = 0; j < c.nblk && ok; ++j) {
+          const int g = g0 + j;
+          const int sk = g % NSK;
+          if (j > 0) {
+            ok = ready_v(g - 1, j - 1, c.kv_len) && pv(0, g - 1, j - 1, n);
+            if (!ok) break;
+          }
+          ok = wait_warp(&bar[(kRope ? B_KREADY : B_KFULL) + sk],
+                         (g / NSK) & 1, abort_flag, status);
           if (!ok) break;
-        }
-        ok = wait_warp(&bar[(kRope ? B_KREADY : B_KFULL) + sk], (j / NSK) & 1,
-                       abort_flag, status);
-        if (!ok) break;
-        tc_fence_after();
-        issue_s(0, j);
-        if (j > 0) {
-          ok = pv(1, j - 1);
-          if (!ok) break;
-          commit(&bar[B_VEMPTY + (j - 1) % NSV]);
-        }
-        issue_s(1, j);
-        commit(&bar[B_KEMPTY + sk]);
-      }
-      if (ok) {
-        const int i = nblk - 1;
-        ok = ready_v(i) && pv(0, i);
-        if (ok) {
-          commit(&bar[B_OFINAL + 0]);
-          ok = pv(1, i);
+          tc_fence_after();
+          issue_s(0, g);
+          if (j > 0) {
+            ok = pv(1, g - 1, j - 1, n);
+            if (!ok) break;
+            commit(&bar[B_VEMPTY + (g - 1) % NSV]);
+          }
+          issue_s(1, g);
+          // the item's last S: the Q buffer is free once these are done
+          if (j == c.nblk - 1) commit(&bar[B_QEMPTY]);
+          commit(&bar[B_KEMPTY + sk]);
         }
         if (ok) {
-          commit(&bar[B_OFINAL + 1]);
-          commit(&bar[B_VEMPTY + i % NSV]);
+          const int jl = c.nblk - 1, g = g0 + jl;
+          ok = ready_v(g, jl, c.kv_len) && pv(0, g, jl, n);
+          if (ok) {
+            commit(&bar[B_OFINAL + 0]);
+            ok = pv(1, g, jl, n);
+          }
+          if (ok) {
+            commit(&bar[B_OFINAL + 1]);
+            commit(&bar[B_VEMPTY + g % NSV]);
+          }
         }
+        g0 += c.nblk;
       }
       // Drain every MMA before tensor memory is released.
       commit(&bar[B_DRAIN]);
@@ -531,24 +595,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (kRope) {
       // -------------------------------------------------------------- RoPE --
       const int tr = threadIdx.x - 320;  // 0..63
-      bool ok = wait_warp(&bar[B_QFULL], 0, abort_flag, status);
-      if (ok) {
+      bool ok = true;
+      int g0 = 0;
+      for (int it = blockIdx.x, n = 0;
+           it < (kPersist ? args.items : blockIdx.x + 1) && ok;
+           it += gridDim.x, ++n) {
+        const Item c = item_of(args, it);
+        ok = wait_warp(&bar[B_QFULL], n & 1, abort_flag, status);
+        if (!ok) break;
         for (int rr = tr; rr < QT * BM; rr += kRopeThreads) {
-          const int n = q0 + rr;
-          if (n < args.Lq) rope_row(sQ + (rr >> 7) * TILE, rr & 127, n, args);
+          const int tok = c.q0 + rr;
+          if (tok < args.Lq)
+            rope_row(sQ + (rr >> 7) * TILE, rr & 127, tok, args);
         }
         fence_proxy_async_smem();
         mbar_arrive(&bar[B_QREADY]);
-      }
-      for (int j = 0; j < nblk && ok; ++j) {
-        const int sk = j % NSK;
-        ok = wait_warp(&bar[B_KFULL + sk], (j / NSK) & 1, abort_flag, status);
-        if (!ok) break;
-        for (int rr = tr; rr < BN; rr += kRopeThreads)
-          if (j * BN + rr < kv_len)
-            rope_row(sK + sk * TILE, rr, j * BN + rr, args);
-        fence_proxy_async_smem();
-        mbar_arrive(&bar[B_KREADY + sk]);
+        for (int j = 0; j < c.nblk && ok; ++j) {
+          const int g = g0 + j, sk = g % NSK;
+          ok = wait_warp(&bar[B_KFULL + sk], (g / NSK) & 1, abort_flag,
+                         status);
+          if (!ok) break;
+          for (int rr = tr; rr < BN; rr += kRopeThreads)
+            if (j * BN + rr < c.kv_len)
+              rope_row(sK + sk * TILE, rr, j * BN + rr, args);
+          fence_proxy_async_smem();
+          mbar_arrive(&bar[B_KREADY + sk]);
+        }
+        g0 += c.nblk;
       }
     }
   } else {
@@ -561,112 +634,128 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t s_col = lane_base + t * 128;
     const uint32_t o_col = lane_base + TM_O + t * 128;
     const float c2 = args.scale_log2;
-    // Keys this row may see: all kv_len, or its block-causal limit.
-    int row_lim = kv_len;
-    if (args.chunk && q0 + t * BM + r < args.Lq) {
-      const int a = q0 + t * BM + r + args.q_offset;
-      row_lim = min(args.Lk, (a / args.chunk + 1) * args.chunk);
-    }
-    float m_run = -INFINITY;
-    float l_run = 0.f;
     bool ok = true;
-    for (int j = 0; j < nblk; ++j) {
-      ok = wait_warp(&bar[B_SFULL + t], j & 1, abort_flag, status);
-      if (!ok) break;
-      tc_fence_after();
-      float s[BN];
-      static_assert(BN == 128, "one 128-column TMEM load per score row");
-      tmem_ld128(s_col, s);
-      tmem_ld_wait128(s);
-      const int lim = row_lim - j * BN;  // valid keys of this row here
-      // warp-uniform: any masked row sends the warp down the exact path
-      const bool masked = __any_sync(0xffffffffu, lim < BN);
-      if (masked) {
-#pragma unroll
-        for (int c = 0; c < BN; ++c)
-          if (c >= lim) s[c] = -INFINITY;
+    int g0 = 0;
+    for (int it = blockIdx.x, n = 0;
+         it < (kPersist ? args.items : blockIdx.x + 1) && ok;
+         it += gridDim.x, ++n) {
+      const Item cur = item_of(args, it);
+      // Keys this row may see: all kv_len, or its block-causal limit.
+      int row_lim = cur.kv_len;
+      if (args.chunk && cur.q0 + t * BM + r < args.Lq) {
+        const int a = cur.q0 + t * BM + r + args.q_offset;
+        row_lim = min(args.Lk, (a / args.chunk + 1) * args.chunk);
       }
-      const float mx = (masked ? rowmax_masked<BN>(s) : rowmax<BN>(s)) * c2;
-      if (j == 0) {
-        m_run = mx;
-      } else {
-        // Keep the running max unless some row's max grew by more than 2^8:
-        // exponents then stay <= 8 (p <= 256, exact after the final O / l).
-        // Otherwise rescale O in TMEM first.  S_t(j) complete implies
-        // PV_t(j-1) complete (issued before it), so O holds exactly blocks
-        // 0..j-1 here; the first part's arrival orders these stores before
-        // PV_t(j).
-        const bool need = mx > m_run + RESCALE_LOG2;
-        if (__any_sync(0xffffffffu, need)) {
-          const float m_new = need ? mx : m_run;
-          const float alpha = ex2(m_run - m_new);
+      float m_run = -INFINITY;
+      float l_run = 0.f;
+      for (int j = 0; j < cur.nblk; ++j) {
+        ok = wait_warp(&bar[B_SFULL + t], (g0 + j) & 1, abort_flag, status);
+        if (!ok) break;
+        tc_fence_after();
+        float s[BN];
+        static_assert(BN == 128, "one 128-column TMEM load per score row");
+        tmem_ld128(s_col, s);
+        tmem_ld_wait128(s);
+        const int lim = row_lim - j * BN;  // valid keys of this row here
+        // warp-uniform: any masked row sends the warp down the exact path
+        const bool masked = __any_sync(0xffffffffu, lim < BN);
+        if (masked) {
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            float o[32];
-            tmem_ld32(o_col + c * 32, o);
-            tmem_ld_wait32(o);
-#pragma unroll
-            for (int e = 0; e < 32; e += 2) {
-              const float2 v =
-                  ffma2(make_float2(o[e], o[e + 1]),
-                        make_float2(alpha, alpha), make_float2(0.f, 0.f));
-              o[e] = v.x;
-              o[e + 1] = v.y;
-            }
-            tmem_st32(o_col + c * 32, o);
-          }
-          l_run *= alpha;
-          m_run = m_new;
+          for (int c = 0; c < BN; ++c)
+            if (c >= lim) s[c] = -INFINITY;
         }
+        const float mx = (masked ? rowmax_masked<BN>(s) : rowmax<BN>(s)) * c2;
+        if (j == 0) {
+          m_run = mx;
+        } else {
+          // Keep the running max unless some row's max grew by more than 2^8:
+          // exponents then stay <= 8 (p <= 256, exact after the final O / l).
+          // Otherwise rescale O in TMEM first.  S_t(j) complete implies
+          // PV_t(j-1) complete (issued before it), so O holds exactly blocks
+          // 0..j-1 here; the first part's arrival orders these stores before
+          // PV_t(j).
+          const bool need = mx > m_run + RESCALE_LOG2;
+          if (__any_sync(0xffffffffu, need)) {
+            const float m_new = need ? mx : m_run;
+            const float alpha = ex2(m_run - m_new);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              float o[32];
+              tmem_ld32(o_col + c * 32, o);
+              tmem_ld_wait32(o);
+#pragma unroll
+              for (int e = 0; e < 32; e += 2) {
+                const float2 v =
+                    ffma2(make_float2(o[e], o[e + 1]),
+                          make_float2(alpha, alpha), make_float2(0.f, 0.f));
+                o[e] = v.x;
+                o[e + 1] = v.y;
+              }
+              tmem_st32(o_col + c * 32, o);
+            }
+            l_run *= alpha;
+            m_run = m_new;
+          }
+        }
+        float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                         make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        // Publish P part by part: the MMA issuer starts P V on the first keys
+        // while the rest are exponentiated.
+        auto publish = [&](int part) {
+          tmem_st_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar[B_PPART + t * NPART + part]);
+        };
+        constexpr int CPP = BN / 32 / NPART;  // 32-key chunks per part
+#pragma unroll
+        for (int part = 0; part < NPART; ++part) {
+          if (masked)
+            exp_store_chunks<false>(s, c2, m_run, s_col, acc, part * CPP,
+                                    (part + 1) * CPP);
+          else
+            exp_store_chunks<true>(s, c2, m_run, s_col, acc, part * CPP,
+                                   (part + 1) * CPP);
+          publish(part);
+        }
+        const float2 tsum = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
+        l_run += tsum.x + tsum.y;
       }
-      float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                       make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-      // Publish P part by part: the MMA issuer starts P V on the first keys
-      // while the rest are exponentiated.
-      auto publish = [&](int part) {
-        tmem_st_wait();
+      g0 += cur.nblk;
+      if (ok) ok = wait_warp(&bar[B_OFINAL + t], n & 1, abort_flag, status);
+      if (ok) {
+        tc_fence_after();
+        // Recompute the item's coordinates here instead of holding them in
+        // registers through the key-block loop.
+        int it_e = it;
+        asm volatile("" : "+r"(it_e));
+        const Item ce = item_of(args, it_e);
+        const float inv = 1.0f / l_run;
+        const int row = ce.q0 + t * BM + r;
+        __nv_bfloat16* orow =
+            args.o + ((static_cast<int64_t>(ce.b) * args.Lq + row) *
+                          args.heads + ce.head) * HD;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          float o[32];
+          tmem_ld32(o_col + c * 32, o);
+          tmem_ld_wait32(o);
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            pk[e] = pack_bf16x2(o[2 * e] * inv, o[2 * e + 1] * inv);
+          if (row < args.Lq) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2],
+                                  pk[4 * e + 3]);
+          }
+        }
+        // O_t has been read: the next item's first P V may overwrite it
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bar[B_PPART + t * NPART + part]);
-      };
-      constexpr int CPP = BN / 32 / NPART;  // 32-key chunks per part
-#pragma unroll
-      for (int part = 0; part < NPART; ++part) {
-        if (masked)
-          exp_store_chunks<false>(s, c2, m_run, s_col, acc, part * CPP,
-                                  (part + 1) * CPP);
-        else
-          exp_store_chunks<true>(s, c2, m_run, s_col, acc, part * CPP,
-                                 (part + 1) * CPP);
-        publish(part);
-      }
-      const float2 tsum = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
-      l_run += tsum.x + tsum.y;
-    }
-    if (ok) ok = wait_warp(&bar[B_OFINAL + t], 0, abort_flag, status);
-    if (ok) {
-      tc_fence_after();
-      const float inv = 1.0f / l_run;
-      const int row = q0 + t * BM + r;
-      __nv_bfloat16* orow =
-          args.o + ((static_cast<int64_t>(b) * args.Lq + row) * args.heads +
-                    head) * HD;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float o[32];
-        tmem_ld32(o_col + c * 32, o);
-        tmem_ld_wait32(o);
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e)
-          pk[e] = pack_bf16x2(o[2 * e] * inv, o[2 * e + 1] * inv);
-        if (row < args.Lq) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2],
-                                pk[4 * e + 3]);
-        }
+        if (lane == 0) mbar_arrive(&bar[B_OFREE + t]);
       }
     }
   }
@@ -746,9 +835,9 @@ int make_map(CUtensorMap* m, const void* base, int B, int L, int heads) {
   return r == CUDA_SUCCESS ? WAN_OK : WAN_EINVAL;
 }
 
-template <int kRope>
+template <int kRope, int kPersist>
 int launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-           const AttnArgs& a, int B, cudaStream_t s) {
+           AttnArgs a, int B, cudaStream_t s) {
   static std::mutex mu;
   static int state[64];  // 0 unknown, 1 ready, 2 unusable
   int dev = 0;
@@ -761,13 +850,14 @@ int launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
       // to launch if the compiled register count cannot fund the split
       // (the .inc would otherwise wait forever).
       cudaFuncAttributes fa;
-      if (cudaFuncGetAttributes(&fa, attn_fwd_kernel<kRope>) != cudaSuccess)
+      if (cudaFuncGetAttributes(&fa, attn_fwd_kernel<kRope, kPersist>) !=
+          cudaSuccess)
         return WAN_ECUDA;
       const int need = 8 * 32 * kSoftmaxRegs + 4 * 32 * kOtherRegs;
       if (fa.numRegs * kThreads < need) {
         state[dev] = 2;
       } else if (cudaFuncSetAttribute(
-                     attn_fwd_kernel<kRope>,
+                     attn_fwd_kernel<kRope, kPersist>,
                      cudaFuncAttributeMaxDynamicSharedMemorySize,
                      SMEM_DYN) != cudaSuccess) {
         return WAN_ECUDA;
@@ -777,8 +867,23 @@ int launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
     }
     if (state[dev] != 1) return WAN_EUNSUPPORTED;
   }
-  dim3 grid((a.Lq + QT * BM - 1) / (QT * BM), a.heads, B);
-  attn_fwd_kernel<kRope><<<grid, kThreads, SMEM_DYN, s>>>(mq, mk, mv, a);
+  a.n_tiles_x = (a.Lq + QT * BM - 1) / (QT * BM);
+  const int64_t items = static_cast<int64_t>(a.n_tiles_x) * a.heads * B;
+  if (items > INT32_MAX) return WAN_EINVAL;
+  a.items = static_cast<int>(items);
+  // One CTA per item, except cross-attention: its items are short (a few
+  // key blocks), so one persistent CTA per SM walks them and loads the next
+  // item's Q while the current one drains.
+  int grid = a.items;
+  if (kPersist) {
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+        cudaSuccess)
+      return WAN_ECUDA;
+    grid = a.items < sms ? a.items : sms;
+  }
+  attn_fwd_kernel<kRope, kPersist><<<grid, kThreads, SMEM_DYN, s>>>(mq, mk, mv,
+                                                                     a);
   return cudaGetLastError() == cudaSuccess ? WAN_OK : WAN_ECUDA;
 }
 
@@ -835,8 +940,8 @@ int wan_self_attn(const void* q, const void* k, const void* v, void* o,
   a.cross = 0;
   a.chunk = 0;
   a.q_offset = 0;
-  return d_table ? launch<1>(mq, mk, mv, a, B, as_stream(s))
-                 : launch<0>(mq, mk, mv, a, B, as_stream(s));
+  return d_table ? launch<1, 0>(mq, mk, mv, a, B, as_stream(s))
+                 : launch<0, 0>(mq, mk, mv, a, B, as_stream(s));
 }
 
 int wan_block_causal_attn(const void* q, const void* k, const void* v,
@@ -867,7 +972,7 @@ int wan_block_causal_attn(const void* q, const void* k, const void* v,
   a.cross = 0;
   a.chunk = chunk_tokens;
   a.q_offset = q_offset;
-  return launch<0>(mq, mk, mv, a, B, as_stream(s));
+  return launch<0, 0>(mq, mk, mv, a, B, as_stream(s));
 }
 
 int wan_cross_attn(const void* q, const void* k_ctx, const void* v_ctx,
@@ -898,7 +1003,7 @@ int wan_cross_attn(const void* q, const void* k_ctx, const void* v_ctx,
   a.chunk = 0;
   a.q_offset = 0;
   for (int i = 0; i < B; ++i) a.lens[i] = ctx_lens[i];
-  return launch<0>(mq, mk, mv, a, B, as_stream(s));
+  return launch<0, 1>(mq, mk, mv, a, B, as_stream(s));
 }
 
 int wan_wait_selftest(int arrive, void* s) {
