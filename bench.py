@@ -47,7 +47,7 @@ def parse():
                    help="skip the HBM-bound kernel rooflines")
     p.add_argument("--no-causal", action="store_true",
                    help="skip the block-causal attention measurement")
-    p.add_argument("--hbm-elems", type=int, default=1 << 28,
+    p.add_argument("--hbm-elems", type=int, default=1 << 30,
                    help="fp32 elements per buffer of the fm_step roofline")
     p.add_argument("--cpu-rows", type=int, default=4096,
                    help="query rows of one head timed on the oracle")
@@ -224,10 +224,10 @@ def job_throughput(world, flops_per_step, steps, max_ms):
     return world * flops_per_step * steps / (max_ms / 1e3) / 1e12
 
 
-def hbm_rooflines(dev, g, L, H, n_lat, peak_gbs, n=1 << 28, reps=20):
+def hbm_rooflines(dev, g, L, H, n_lat, peak_gbs, n=1 << 30, reps=20):
     """Achieved bandwidth of the HBM-bound kernels, timed alone with CUDA
     events: the fused CFG + Euler step and the fused UniPC stop on n-element
-    fp32 buffers (default 2^28: 4 GiB / 9 GiB of traffic per call, far above
+    fp32 buffers (default 2^30: 16 GiB / 36 GiB of traffic per call, far above
     L2), the RoPE, QK-Norm + RoPE, AdaLN and gated-residual passes on the
     workload's tensors; plus the Euler step on the workload's own latent,
     timed cold (L2 flushed by a 512 MiB write before every call)."""
