@@ -86,3 +86,42 @@ def test_480p_17f_frame_chunks():
     want = oattn.block_causal_attention(f64(q), f64(k), f64(v), scale_for(),
                                         chunk)
     assert_attn_close(got, want, "block-causal 7800")
+
+
+# ---- the launch configuration bench.py times: 480p-165f, 42 x 30 x 52 =
+# 65,520 tokens, 40 heads, chunks of 3 latent frames (4,680 tokens).  The
+# oracle evaluates sampled rows on a sample of heads (heads are independent).
+FULL_L, FULL_H, FULL_CHUNK = 65520, 40, 4680
+HEADS = np.array([0, 13, 27, 39])
+
+
+def _full_qkv():
+    return _qkv(1, FULL_L, FULL_L, FULL_H, 900)
+
+
+def _rows(n_total, seed, extra=()):
+    rows = inputs.sample_rows(n_total, 96, seed).numpy()
+    return np.unique(np.concatenate([rows, np.asarray(extra, np.int64)]))
+
+
+def test_full_sequence_480p_165f_sampled():
+    q, k, v = _full_qkv()
+    got = _run(q, k, v, FULL_CHUNK)
+    # rows on both sides of chunk boundaries and in the first chunk
+    rows = _rows(FULL_L, 91, [1, 4679, 4680, 32759, 32760, 60839, 60840])
+    want = oattn.block_causal_attention(
+        f64(q[:, :, HEADS]), f64(k[:, :, HEADS]), f64(v[:, :, HEADS]),
+        scale_for(128), FULL_CHUNK, 0, rows)
+    assert_attn_close(got[:, rows][:, :, HEADS], want, "480p-165f full")
+
+
+def test_kv_cache_last_chunk_480p_165f_sampled():
+    q, k, v = _full_qkv()
+    q0 = FULL_L - FULL_CHUNK
+    ql = q[:, q0:].contiguous()
+    got = _run(ql, k, v, FULL_CHUNK, q0)
+    rows = _rows(FULL_CHUNK, 92, [1, FULL_CHUNK - 2])
+    want = oattn.block_causal_attention(
+        f64(ql[:, :, HEADS]), f64(k[:, :, HEADS]), f64(v[:, :, HEADS]),
+        scale_for(128), FULL_CHUNK, q0, rows)
+    assert_attn_close(got[:, rows][:, :, HEADS], want, "480p-165f KV step")
