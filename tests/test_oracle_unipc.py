@@ -181,3 +181,59 @@ def test_sigma_one_is_the_limit():
         (1e-3, 1e-6, 1e-10, 1e-15)]
     assert all(g1 > g2 for g1, g2 in zip(gaps, gaps[1:])), gaps
     assert gaps[-1] <= 2e-6
+
+
+# ---- planted mistakes: each must break one of the pins above ------------
+
+def _predictor_error():
+    a, b = _rand(16, 21), _rand(16, 22)
+    m_of = lambda lam: a + b * lam
+    sig = np.array([0.9, 0.7, 0.45, 0.2, 0.0])
+    x_i = _rand(16, 23)
+    m = {k: m_of(unipc.log_snr(sig[k])) for k in (0, 1)}
+    got = unipc.predictor(x_i, m, sig, 1)
+    want = _ode_solution(x_i, sig[1], sig[2], m_of)
+    return np.max(np.abs(got - want))
+
+
+def _corrector_error():
+    a, b, c = _rand(16, 31), _rand(16, 32), _rand(16, 33)
+    m_of = lambda lam: a + b * lam + c * lam ** 2
+    sig = np.array([0.95, 0.8, 0.6, 0.35, 0.0])
+    x_prev = _rand(16, 34)
+    m = {k: m_of(unipc.log_snr(sig[k])) for k in (0, 1, 2)}
+    got = unipc.corrector(x_prev, m, sig, 2)
+    want = _ode_solution(x_prev, sig[1], sig[2], m_of)
+    return np.max(np.abs(got - want))
+
+
+def test_pins_hold_unplanted():
+    assert _predictor_error() < 1e-9
+    assert _corrector_error() < 1e-9
+
+
+def test_planted_phi_order_mistake_is_caught(monkeypatch):
+    right = unipc.phi_q
+    monkeypatch.setattr(unipc, "phi_q", lambda k, h: right(k + 1, h)
+                        if k >= 1 else right(k, h))
+    assert _predictor_error() > 1e-4
+
+
+def test_planted_dropped_new_point_is_caught(monkeypatch):
+    right = unipc.exponential_update
+
+    def drop_last(x_s, sigma_s, sigma_t, m_s, diffs):
+        return right(x_s, sigma_s, sigma_t, m_s, diffs[:-1])
+    monkeypatch.setattr(unipc, "exponential_update", drop_last)
+    assert _corrector_error() > 1e-4
+
+
+def test_planted_clean_estimate_sign_is_caught(monkeypatch):
+    monkeypatch.setattr(unipc._step, "x0_estimate",
+                        lambda x, v, s: np.asarray(x, np.float64)
+                        + float(s) * np.asarray(v, np.float64))
+    sig = schedule.sigmas(40, 12.0)
+    x, vc = _rand(64, 1), _rand(64, 2)
+    x1, _, _ = unipc.unipc_step(x, None, None, None, vc, None, 1.0, sig, 0)
+    want = step.fm_step(x, vc, None, 1.0, sig[0], sig[1])
+    assert np.max(np.abs(x1 - want)) > 1e-3
