@@ -8,6 +8,8 @@ import math
 
 import numpy as np
 import pytest
+from hypothesis import given, settings
+from hypothesis import strategies as hst
 
 from oracle import schedule, unipc
 from video_diffusion_transformer_self_b200 import build, wan
@@ -117,3 +119,23 @@ def test_rejects(lib):
         == wan.WAN_EINVAL
     assert st(None, None, None, None, None, None, None, 1.0, 0, arr, 4, 2,
               None) == wan.WAN_OK  # empty: nothing to do
+
+
+@hst.composite
+def schedules(draw):
+    n = draw(hst.integers(1, 30))
+    shift = draw(hst.floats(0.5, 20.0))
+    smax = draw(hst.sampled_from([1.0, 0.999, 0.95, 0.7]))
+    return schedule.sigmas(n, shift, smax)
+
+
+@settings(max_examples=40, deadline=None)
+@given(schedules(), hst.data())
+def test_coefficients_match_oracle_random_schedules(sig, data):
+    build.build()
+    n = len(sig) - 1
+    i = data.draw(hst.integers(0, n - 1))
+    got = wan.unipc_coeffs(sig, i)
+    want = oracle_coeffs(sig, i)
+    for key, w in want.items():
+        assert got[key] == pytest.approx(w, rel=1e-10, abs=1e-13), (key, i)
