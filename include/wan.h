@@ -1,14 +1,18 @@
 /*
  * wan.h -- C ABI of libwan, the B200 (sm_100a) hot path of the Wan2.1 /
  * Wan2.2 video diffusion transformer: 3D RoPE, full spatio-temporal
- * self-attention, length-masked cross-attention to text, and the shifted
- * sigma schedule with the fused CFG + Euler flow step.
+ * self-attention, length-masked cross-attention to text, block-causal
+ * (chunked, KV-cache) attention, the block prologue / epilogue (AdaLN
+ * modulate, QK-Norm + RoPE, gated residual), the shifted sigma schedule
+ * with the fused CFG + Euler flow step, the fused UniPC order-2 sampler
+ * stop, and the layout moves around the Ulysses all-to-all.
  *
  * Sources (cited by page and section):
  *   "Wan2.2 source reading" -- blog.leeguoo.com, "動画生成の勘定を明らかにする：
  *       Wan2.2 ソースコード精読";
  *   "Wan paper explainer"   -- 0h-n0.github.io, "論文解説: Wan - 大規模オープン
- *       ソース動画生成モデルのアーキテクチャと訓練".
+ *       ソース動画生成モデルのアーキテクチャと訓練";
+ *   "Long-video survey"     -- the atlascloud.ai long-video generation blog.
  *
  * Conventions shared by every call
  * --------------------------------
