@@ -8,7 +8,7 @@ self-attention input is ``norm1(x) * (1 + e[1]) + e[0]`` and the block output
 "3D RoPE", last paragraph: in the self-attention, q and k each go through an
 RMSNorm (QK-Norm) after their linear layers, before the rotation.
 
-Readings (listed in DESIGN.md):
+Readings taken where the page is silent:
 
 * norm1 is a LayerNorm over the model dim without its own affine weights
   (the modulation supplies scale and shift), eps = 1e-6;

@@ -10,7 +10,7 @@ rotation is applied to q and k as a complex multiplication, in float64 with
 autocast disabled.  The section states that after rotation q.k depends only
 on the coordinate difference of the two tokens (translation invariance).
 
-Readings where the page is silent (listed again in the design doc):
+Readings where the page is silent:
 
 * base theta = 10000 (the workloads state it; the page does not print the
   body of ``rope_params``);

@@ -11,7 +11,7 @@ half of the points fall at t > 926 and the first timesteps (printed as
 integers) are 999, 997, 995, 993, 990, 988.  Ch. 6 ("boundary and shift"):
 with boundary 0.875, 26 of the 40 steps have t >= 875 and 14 fall below.
 
-Readings (listed in DESIGN.md):
+Readings taken where the page is silent:
 
 * "laid uniformly" is s_i = s_max * (1 - i / N) for i = 0 .. N-1, with
   s_max = 1 by default; the printed list is reproduced with s_max = 0.999

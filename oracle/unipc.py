@@ -13,8 +13,8 @@ clean estimate ``x0_pred = sample - sigma * model_output``.
 The pages give no coefficient, so the steps below follow the published UniPC
 method (Zhao et al., "UniPC: A Unified Predictor-Corrector Framework for Fast
 Sampling of Diffusion Models", 2023) in its data-prediction form, with the
-coefficients solved exactly from its order conditions.  Readings (listed in
-DESIGN.md):
+coefficients solved exactly from its order conditions.  Readings taken
+where the pages are silent:
 
 * alpha = 1 - sigma and lambda = log(alpha / sigma), the half log-SNR of the
   straight path; lambda(1) = -inf and lambda(0) = +inf are taken as limits;

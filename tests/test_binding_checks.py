@@ -56,3 +56,86 @@ def test_host_calls_validate():
         wan.unipc_coeffs([1.0, 0.5, 0.5, 0.0], 1)       # not decreasing
     with pytest.raises(wan.WanError):
         wan.token_grid(80, 720, 1280)                   # frames not 4n + 1
+
+
+# ---- shapes and sizes: checked before the device, so CPU tensors with a
+# mismatched shape are refused for the shape (the kernels build their tensor
+# maps and strides from q's heads, the grid's F*H*W and k's length, so any
+# mismatch would read or write past an allocation).
+
+def test_self_attn_rejects_shape_mismatch():
+    g = wan.grid(2, 4, 4)
+    q = _bf16(1, 32, 2, 128)
+    with pytest.raises(ValueError, match="shape"):
+        wan.self_attn(q, _bf16(1, 32, 3, 128), q, q, g)     # k heads
+    with pytest.raises(ValueError, match="shape"):
+        wan.self_attn(q, q, _bf16(1, 31, 2, 128), q, g)     # v length
+    with pytest.raises(ValueError, match="shape"):
+        wan.self_attn(q, q, q, _bf16(2, 32, 2, 128), g)     # o batch
+    with pytest.raises(ValueError, match="tokens"):
+        wan.self_attn(q, q, q, q, wan.grid(2, 4, 5))        # L != F*H*W
+    with pytest.raises(ValueError, match="bytes"):
+        wan.self_attn(q, q, q, q, g, table=torch.zeros(16, dtype=torch.uint8))
+
+
+def test_cross_and_causal_reject_shape_mismatch():
+    q = _bf16(2, 40, 2, 128)
+    kc = _bf16(2, 16, 2, 128)
+    with pytest.raises(ValueError, match="shape"):
+        wan.cross_attn(q, kc, _bf16(2, 15, 2, 128), q.clone(), [3, 4])
+    with pytest.raises(ValueError, match="shape"):
+        wan.cross_attn(q, _bf16(1, 16, 2, 128), _bf16(1, 16, 2, 128),
+                       q.clone(), [3, 4])                      # k batch
+    with pytest.raises(ValueError, match="shape"):
+        wan.cross_attn(q, _bf16(2, 16, 4, 128), _bf16(2, 16, 4, 128),
+                       q.clone(), [3, 4])                      # k heads
+    with pytest.raises(ValueError, match="shape"):
+        wan.cross_attn(q, kc, kc.clone(), _bf16(2, 41, 2, 128), [3, 4])
+    with pytest.raises(ValueError, match="lengths"):
+        wan.cross_attn(q, kc, kc.clone(), q.clone(), [3])
+    k = _bf16(2, 80, 2, 128)
+    with pytest.raises(ValueError, match="shape"):
+        wan.block_causal_attn(q, k, _bf16(2, 79, 2, 128), q.clone(), 8)
+    with pytest.raises(ValueError, match="shape"):
+        wan.block_causal_attn(q, k, k.clone(), _bf16(2, 40, 1, 128), 8)
+
+
+def test_rope_and_block_kernels_reject_sizes():
+    g = wan.grid(2, 4, 4)
+    q = _bf16(1, 32, 2, 128)
+    with pytest.raises(ValueError, match="shape"):
+        wan.rope3d_qk(q, _bf16(1, 32, 1, 128), g, torch.zeros(4096,
+                                                             dtype=torch.uint8))
+    with pytest.raises(ValueError, match="tokens"):
+        wan.rope3d_qk(q, q.clone(), wan.grid(1, 4, 4),
+                      torch.zeros(4096, dtype=torch.uint8))
+    with pytest.raises(ValueError, match="bytes"):
+        wan.rope3d_qk(q, q.clone(), g, torch.zeros(8, dtype=torch.uint8))
+    with pytest.raises(ValueError, match="elements"):
+        wan.qk_norm_rope(q, q.clone(), torch.zeros(255), torch.zeros(256), g,
+                         torch.zeros(4096, dtype=torch.uint8))
+    x = torch.zeros(1, 2, 8)
+    with pytest.raises(ValueError, match="size"):
+        wan.gated_residual(x, _bf16(1, 2, 7), torch.zeros(1, 8))
+    with pytest.raises(ValueError, match="elements"):
+        wan.gated_residual(x, _bf16(1, 2, 8), torch.zeros(1, 7))
+    with pytest.raises(ValueError, match="elements"):
+        wan.adaln_modulate(x, torch.zeros(1, 8), torch.zeros(1, 8),
+                           _bf16(1, 2, 7))
+    with pytest.raises(ValueError, match="elements"):
+        wan.adaln_modulate(x, torch.zeros(1, 9), torch.zeros(1, 8),
+                           _bf16(1, 2, 8))
+    with pytest.raises(ValueError, match="elements"):
+        wan.fm_step(torch.zeros(16), torch.zeros(15), None, 1.0, 1.0, 0.9)
+    with pytest.raises(ValueError, match="elements"):
+        wan.fm_step(torch.zeros(16), torch.zeros(16), torch.zeros(17), 1.0,
+                    1.0, 0.9)
+
+
+def test_right_shapes_on_cpu_fail_only_for_the_device():
+    g = wan.grid(2, 4, 4)
+    q = _bf16(1, 32, 2, 128)
+    with pytest.raises(ValueError, match="CUDA"):
+        wan.self_attn(q, q.clone(), q.clone(), q.clone(), g)
+    with pytest.raises(ValueError, match="CUDA"):
+        wan.fm_step(torch.zeros(16), torch.zeros(16), None, 1.0, 1.0, 0.9)

@@ -129,12 +129,63 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
+# Argument checks run in this order: dtype / rank / layout, then shapes and
+# sizes against each other, then the device (every tensor on one CUDA
+# device), all before the library is called.
+
+
 def _bf16_bl(t, name):
     import torch
-    if t.dtype != torch.bfloat16 or t.dim() != 4 or not t.is_contiguous() \
-            or not t.is_cuda:
-        raise ValueError("%s must be a contiguous CUDA bf16 [B, L, heads, d]"
-                         " tensor" % name)
+    if t.dtype != torch.bfloat16 or t.dim() != 4 or not t.is_contiguous():
+        raise ValueError("%s must be a contiguous bf16 [B, L, heads, d] "
+                         "tensor" % name)
+
+
+def _on_cuda(*named):
+    """Every given (name, tensor) pair (None skipped) is a CUDA tensor, all
+    on the same device."""
+    for name, t in named:
+        if t is not None and not t.is_cuda:
+            raise ValueError("%s must be a CUDA tensor" % name)
+    devs = {t.device for _, t in named if t is not None}
+    if len(devs) > 1:
+        raise ValueError("tensors on different devices: %s" % ", ".join(
+            "%s on %s" % (name, t.device) for name, t in named
+            if t is not None))
+
+
+def _shape_is(t, shape, name):
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError("%s has shape %s, expected %s"
+                         % (name, tuple(t.shape), tuple(shape)))
+
+
+def _grid_tokens(g):
+    return int(g.F) * int(g.H) * int(g.W)
+
+
+def _check_table(table, g, head_dim, name="table"):
+    """A RoPE table must be a contiguous CUDA tensor of at least
+    rope3d_table_bytes(g) bytes (the kernels read that many)."""
+    if table is None:
+        return
+    if not table.is_contiguous():
+        raise ValueError("%s must be a contiguous tensor" % name)
+    need = rope3d_table_bytes(g, head_dim)
+    if need == 0:
+        raise ValueError("grid %r has no RoPE table" % (g,))
+    if table.numel() * table.element_size() < need:
+        raise ValueError("%s holds %d bytes, grid %r needs %d"
+                         % (name, table.numel() * table.element_size(), g,
+                            need))
+
+
+def _f32_n(t, n, name):
+    """Contiguous fp32 tensor of exactly n elements."""
+    _f32(t, name)
+    if t.numel() != n:
+        raise ValueError("%s has %d elements, expected %d"
+                         % (name, t.numel(), n))
 
 
 # ---------------------------------------------------------------- host ---
@@ -173,6 +224,10 @@ def rope3d_table(g, theta=10000.0, head_dim=128, out=None, stream=None):
         raise WanError(WAN_EINVAL, "wan_rope3d_table_bytes")
     if out is None:
         out = torch.empty(n, dtype=torch.uint8, device="cuda")
+    elif not out.is_contiguous() or out.numel() * out.element_size() < n:
+        raise ValueError("out must be a contiguous tensor of at least %d "
+                         "bytes" % n)
+    _on_cuda(("out", out))
     _check(lib().wan_rope3d_table(g, head_dim, theta, _ptr(out), out.numel(),
                                   _stream(stream)), "wan_rope3d_table")
     return out
@@ -181,7 +236,19 @@ def rope3d_table(g, theta=10000.0, head_dim=128, out=None, stream=None):
 def rope3d_qk(q, k, g, table, stream=None):
     """In-place 3D RoPE of q and k ([B, L, heads, 128] bf16)."""
     t = q if q is not None else k
-    _bf16_bl(t, "q/k")
+    if t is None:
+        raise ValueError("q and k are both None")
+    for name, x in (("q", q), ("k", k)):
+        if x is not None:
+            _bf16_bl(x, name)
+            _shape_is(x, t.shape, name)
+    if t.shape[1] != _grid_tokens(g):
+        raise ValueError("q/k hold %d tokens, grid %r has %d"
+                         % (t.shape[1], g, _grid_tokens(g)))
+    _check_table(table, g, t.shape[3])
+    if table is None:
+        raise ValueError("rope3d_qk needs a table")
+    _on_cuda(("q", q), ("k", k), ("table", table))
     _check(lib().wan_rope3d_qk(_ptr(q), _ptr(k), t.shape[0], g, t.shape[2],
                                t.shape[3], _ptr(table), _stream(stream)),
            "wan_rope3d_qk")
@@ -191,7 +258,13 @@ def self_attn(q, k, v, o, g, table=None, softmax_scale=None, stream=None):
     """o = softmax(rope(q) rope(k)^T * scale) v; RoPE fused if table given."""
     for name, t in (("q", q), ("k", k), ("v", v), ("o", o)):
         _bf16_bl(t, name)
+        _shape_is(t, q.shape, name)
     B, L, H, D = q.shape
+    if L != _grid_tokens(g):
+        raise ValueError("q holds %d tokens, grid %r has %d"
+                         % (L, g, _grid_tokens(g)))
+    _check_table(table, g, D)
+    _on_cuda(("q", q), ("k", k), ("v", v), ("o", o), ("table", table))
     if softmax_scale is None:
         softmax_scale = 1.0 / math.sqrt(D)
     _check(lib().wan_self_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, g, H, D,
@@ -206,7 +279,14 @@ def cross_attn(q, k_ctx, v_ctx, o, ctx_lens, softmax_scale=None,
         _bf16_bl(t, name)
     B, Lq, H, D = q.shape
     Lk = k_ctx.shape[1]
-    lens = (ctypes.c_int32 * B)(*[int(x) for x in ctx_lens])
+    _shape_is(o, q.shape, "o")
+    _shape_is(k_ctx, (B, Lk, H, D), "k_ctx")
+    _shape_is(v_ctx, k_ctx.shape, "v_ctx")
+    ctx_lens = [int(x) for x in ctx_lens]
+    if len(ctx_lens) != B:
+        raise ValueError("%d text lengths for batch %d" % (len(ctx_lens), B))
+    _on_cuda(("q", q), ("k_ctx", k_ctx), ("v_ctx", v_ctx), ("o", o))
+    lens = (ctypes.c_int32 * B)(*ctx_lens)
     if softmax_scale is None:
         softmax_scale = 1.0 / math.sqrt(D)
     _check(lib().wan_cross_attn(_ptr(q), _ptr(k_ctx), _ptr(v_ctx), _ptr(o),
@@ -222,6 +302,10 @@ def block_causal_attn(q, k, v, o, chunk_tokens, q_offset=0,
         _bf16_bl(t, name)
     B, Lq, H, D = q.shape
     Lk = k.shape[1]
+    _shape_is(o, q.shape, "o")
+    _shape_is(k, (B, Lk, H, D), "k")
+    _shape_is(v, k.shape, "v")
+    _on_cuda(("q", q), ("k", k), ("v", v), ("o", o))
     if softmax_scale is None:
         softmax_scale = 1.0 / math.sqrt(D)
     _check(lib().wan_block_causal_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(o),
@@ -233,18 +317,24 @@ def block_causal_attn(q, k, v, o, chunk_tokens, q_offset=0,
 
 def _f32(t, name):
     import torch
-    if t.dtype != torch.float32 or not t.is_contiguous() or not t.is_cuda:
-        raise ValueError("%s must be a contiguous CUDA fp32 tensor" % name)
+    if t.dtype != torch.float32 or not t.is_contiguous():
+        raise ValueError("%s must be a contiguous fp32 tensor" % name)
 
 
 def adaln_modulate(x, shift, scale, out, eps=1e-6, stream=None):
     """out = LayerNorm(x) * (1 + scale[b]) + shift[b]; x fp32 [B, L, D]."""
     import torch
-    for name, t in (("x", x), ("shift", shift), ("scale", scale)):
-        _f32(t, name)
-    if out.dtype != torch.bfloat16 or not out.is_contiguous():
-        raise ValueError("out must be a contiguous bf16 tensor")
+    _f32(x, "x")
+    if x.dim() != 3:
+        raise ValueError("x must be [B, L, D]")
     B, L, D = x.shape
+    _f32_n(shift, B * D, "shift")
+    _f32_n(scale, B * D, "scale")
+    if out.dtype != torch.bfloat16 or not out.is_contiguous() \
+            or out.numel() != B * L * D:
+        raise ValueError("out must be a contiguous bf16 tensor of "
+                         "B * L * D elements")
+    _on_cuda(("x", x), ("shift", shift), ("scale", scale), ("out", out))
     _check(lib().wan_adaln_modulate(_ptr(x), _ptr(shift), _ptr(scale),
                                     _ptr(out), B, L, D, eps,
                                     _stream(stream)), "wan_adaln_modulate")
@@ -253,10 +343,26 @@ def adaln_modulate(x, shift, scale, out, eps=1e-6, stream=None):
 def qk_norm_rope(q, k, wq, wk, g, table, eps=1e-6, stream=None):
     """In place: t = rope3d(RMSNorm_{heads*128}(t) * w) for t in (q, k)."""
     t = q if q is not None else k
-    _bf16_bl(t, "q/k")
-    for name, w in (("wq", wq), ("wk", wk)):
-        if w is not None:
-            _f32(w, name)
+    if t is None:
+        raise ValueError("q and k are both None")
+    for name, x in (("q", q), ("k", k)):
+        if x is not None:
+            _bf16_bl(x, name)
+            _shape_is(x, t.shape, name)
+    if t.shape[1] != _grid_tokens(g):
+        raise ValueError("q/k hold %d tokens, grid %r has %d"
+                         % (t.shape[1], g, _grid_tokens(g)))
+    if table is None:
+        raise ValueError("qk_norm_rope needs a table")
+    _check_table(table, g, t.shape[3])
+    nw = t.shape[2] * t.shape[3]
+    for name, x, w in (("wq", q, wq), ("wk", k, wk)):
+        if x is not None:
+            if w is None:
+                raise ValueError("%s is needed with its tensor" % name)
+            _f32_n(w, nw, name)
+    _on_cuda(("q", q), ("k", k), ("wq", wq), ("wk", wk),
+                 ("table", table))
     _check(lib().wan_qk_norm_rope(_ptr(q), _ptr(k), _ptr(wq), _ptr(wk),
                                   t.shape[0], g, t.shape[2], t.shape[3],
                                   _ptr(table), eps, _stream(stream)),
@@ -265,19 +371,27 @@ def qk_norm_rope(q, k, wq, wk, g, table, eps=1e-6, stream=None):
 
 def gated_residual(x, y, gate, stream=None):
     """x += y * gate[b]; x fp32 [B, L, D], y bf16 [B, L, D], gate [B, D]."""
+    import torch
     _f32(x, "x")
-    _f32(gate, "gate")
+    if x.dim() != 3:
+        raise ValueError("x must be [B, L, D]")
     B, L, D = x.shape
+    _f32_n(gate, B * D, "gate")
+    if y.dtype != torch.bfloat16 or not y.is_contiguous() \
+            or y.numel() != x.numel():
+        raise ValueError("y must be a contiguous bf16 tensor of x's size")
+    _on_cuda(("x", x), ("y", y), ("gate", gate))
     _check(lib().wan_gated_residual(_ptr(x), _ptr(y), _ptr(gate), B, L, D,
                                     _stream(stream)), "wan_gated_residual")
 
 
 def fm_step(x, v_cond, v_uncond, guide, sigma, sigma_next, stream=None):
     """x += (sigma_next - sigma) * (v_uncond + guide (v_cond - v_uncond))."""
-    import torch
-    for t in (x, v_cond) + ((v_uncond,) if v_uncond is not None else ()):
-        if t.dtype != torch.float32 or not t.is_contiguous() or not t.is_cuda:
-            raise ValueError("fm_step tensors must be contiguous CUDA fp32")
+    _f32(x, "x")
+    _f32_n(v_cond, x.numel(), "v_cond")
+    if v_uncond is not None:
+        _f32_n(v_uncond, x.numel(), "v_uncond")
+    _on_cuda(("x", x), ("v_cond", v_cond), ("v_uncond", v_uncond))
     _check(lib().wan_fm_step(_ptr(x), _ptr(v_cond), _ptr(v_uncond), guide,
                              x.numel(), sigma, sigma_next, _stream(stream)),
            "wan_fm_step")
@@ -305,11 +419,14 @@ def unipc_step(x, x_corr, m_prev1, m_prev2, m_out, v_cond, v_uncond, guide,
     for name, t in (("x", x), ("x_corr", x_corr), ("m_out", m_out),
                     ("v_cond", v_cond), ("v_uncond", v_uncond),
                     ("m_prev1", m_prev1), ("m_prev2", m_prev2)):
-        if t is not None and (t.dtype != torch.float32 or not t.is_cuda
+        if t is not None and (t.dtype != torch.float32
                               or not t.is_contiguous()
                               or t.numel() != x.numel()):
-            raise ValueError("%s must be a contiguous CUDA fp32 tensor of "
-                             "x's size" % name)
+            raise ValueError("%s must be a contiguous fp32 tensor of x's "
+                             "size" % name)
+    _on_cuda(("x", x), ("x_corr", x_corr), ("m_out", m_out),
+                 ("v_cond", v_cond), ("v_uncond", v_uncond),
+                 ("m_prev1", m_prev1), ("m_prev2", m_prev2))
     arr, n = _sigma_array(sigmas)
     _check(lib().wan_unipc_step(_ptr(x), _ptr(x_corr), _ptr(m_prev1),
                                 _ptr(m_prev2), _ptr(m_out), _ptr(v_cond),
@@ -320,10 +437,11 @@ def unipc_step(x, x_corr, m_prev1, m_prev2, m_out, v_cond, v_uncond, guide,
 def transpose_blocks(inp, out, a, b, row_bytes, stream=None):
     """out[j][i][:] = inp[i][j][:] (i < a, j < b, rows of row_bytes)."""
     for name, t in (("inp", inp), ("out", out)):
-        if not t.is_cuda or not t.is_contiguous():
-            raise ValueError("%s must be a contiguous CUDA tensor" % name)
+        if not t.is_contiguous():
+            raise ValueError("%s must be a contiguous tensor" % name)
         if t.numel() * t.element_size() < a * b * row_bytes:
             raise ValueError("%s is smaller than a * b * row_bytes" % name)
+    _on_cuda(("inp", inp), ("out", out))
     _check(lib().wan_transpose_blocks(_ptr(inp), _ptr(out), int(a), int(b),
                                       int(row_bytes), _stream(stream)),
            "wan_transpose_blocks")
