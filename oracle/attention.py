@@ -118,16 +118,29 @@ def attend_limited(q, k, v, scale, limits):
 
 
 def block_causal_attention(q, k, v, scale, chunk_tokens, q_offset=0,
-                           rows=None):
-    """Block-causal attention over [B, L, heads, d] tensors (fp64)."""
+                           rows=None, row_block=512):
+    """Block-causal attention over [B, L, heads, d] tensors (fp64).
+
+    Every query of one chunk has the same key limit, so the rows sharing a
+    limit n are evaluated together as plain attention over keys 0 .. n-1
+    (``attend``), in groups of at most ``row_block`` rows; each row is the
+    same definition as ``attend_limited`` gives it.
+    """
     q = np.asarray(q)
     b_, lq, nh, d = q.shape
     lk = np.asarray(k).shape[1]
     lim = block_causal_limits(lq, lk, chunk_tokens, q_offset)
     rows = np.arange(lq) if rows is None else np.asarray(rows)
+    lim_r = lim[rows]
     out = np.empty((b_, rows.shape[0], nh, d), dtype=np.float64)
     for b in range(b_):
         for h in range(nh):
-            out[b, :, h, :] = attend_limited(q[b, rows, h, :], k[b, :, h, :],
-                                             v[b, :, h, :], scale, lim[rows])
+            kh = np.asarray(k[b, :, h, :], dtype=np.float64)
+            vh = np.asarray(v[b, :, h, :], dtype=np.float64)
+            for n in np.unique(lim_r):
+                idx = np.nonzero(lim_r == n)[0]
+                for r0 in range(0, idx.shape[0], row_block):
+                    sel = idx[r0:r0 + row_block]
+                    out[b, sel, h, :] = attend(q[b, rows[sel], h, :],
+                                               kh[:n], vh[:n], scale)
     return out

@@ -215,3 +215,23 @@ def test_block_causal_limits_and_rejects():
         attention.block_causal_limits(5, 8, 4, q_offset=4)
     with pytest.raises(ValueError):
         attention.block_causal_limits(5, 9, 0)
+
+
+def test_block_causal_grouped_rows_equal_row_by_row():
+    # the grouped evaluation (rows sharing a key limit together, in groups
+    # smaller than a chunk) against the plain row-by-row definition, on
+    # sampled rows and a KV-cache offset
+    rng = np.random.default_rng(17)
+    q = rng.standard_normal((2, 90, 3, 8))
+    k = rng.standard_normal((2, 130, 3, 8))
+    v = rng.standard_normal((2, 130, 3, 8))
+    rows = np.array([0, 1, 5, 19, 20, 21, 44, 60, 89])
+    got = attention.block_causal_attention(q, k, v, 0.35, 20, q_offset=40,
+                                           rows=rows, row_block=2)
+    lim = attention.block_causal_limits(90, 130, 20, 40)
+    for b in range(2):
+        for h in range(3):
+            want = attention.attend_limited(q[b, rows, h], k[b, :, h],
+                                            v[b, :, h], 0.35, lim[rows])
+            np.testing.assert_allclose(got[b, :, h], want, rtol=1e-13,
+                                       atol=1e-13)
