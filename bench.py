@@ -41,6 +41,12 @@ def parse():
     p.add_argument("--workload", default="720p-81f")
     p.add_argument("--rope", choices=["fused", "pre"], default="pre")
     p.add_argument("--impl", choices=["wan", "reference"], default="wan")
+    p.add_argument("--parallel", choices=["replicas", "ulysses"],
+                   default="replicas",
+                   help="N > 1: independent problems per rank (replicas), "
+                        "or one problem split by Ulysses head sharding")
+    p.add_argument("--no-points", action="store_true",
+                   help="skip the per-workload self-attention launch points")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-hbm", action="store_true",
@@ -421,6 +427,70 @@ def causal_rooflines(dev, peak_tflops, reps=5):
     return out
 
 
+def attn_points(dev, pk, reps=6):
+    """Self-attention launch alone at the two token counts of the metric:
+    480p-81f (B 2 x 12 heads x 32,760 tokens) and 720p-81f (B 1 x 40 heads
+    x 75,600 tokens), each with Q / K rotated by the stand-alone RoPE pass
+    beforehand ("pre", the step's default) and with the rotation fused into
+    the attention kernel's tile stage ("fused").  CUDA events around `reps`
+    back-to-back launches on the launching stream after 2 warm-up launches;
+    Q, K and V are each larger than L2 at 720p (774 MB) and together above
+    it at 480p (3 x 201 MB).  FLOPs 4 * B * heads * L^2 * 128."""
+    import torch
+
+    from video_diffusion_transformer_self_b200 import wan
+    from video_diffusion_transformer_self_b200.workloads import by_name
+
+    sustained = float(pk.get("bf16_tflops_sustained", 1400.0))
+    burst = float(pk.get("bf16_tflops", 1590.0))
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(6161)
+    stream = torch.cuda.current_stream()
+    out = {}
+    for name in ("480p-81f", "720p-81f"):
+        w = by_name(name)
+        _, g = wan.token_grid(w.frames, w.height, w.width)
+        L, B, H = g.F * g.H * g.W, w.batch, w.heads
+        shape = (B, L, H, 128)
+        q = torch.randn(shape, device=dev, generator=gen).to(torch.bfloat16)
+        k = torch.randn(shape, device=dev, generator=gen).to(torch.bfloat16)
+        v = torch.randn(shape, device=dev, generator=gen).to(torch.bfloat16)
+        o = torch.empty_like(q)
+        table = wan.rope3d_table(g)
+        fl = 4.0 * B * H * L * L * 128
+        point = {"tokens": L, "batch": B, "heads": H, "flops": fl}
+        for mode in ("pre", "fused"):
+            if mode == "pre":
+                wan.rope3d_qk(q, k, g, table)
+
+                def call():
+                    wan.self_attn(q, k, v, o, g)
+            else:
+                def call():
+                    wan.self_attn(q, k, v, o, g, table=table)
+            for _ in range(2):
+                call()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            e0.record(stream)
+            for _ in range(reps):
+                call()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1) / reps
+            tf = fl / (ms / 1e3) / 1e12
+            point[mode] = {"avg_launch_ms": ms, "tflops": tf,
+                           "frac_of_measured_sustained": tf / sustained,
+                           "frac_of_measured_burst": tf / burst,
+                           "frac_of_datasheet_2250": tf / 2250.0}
+        if wan.device_status() != 0:
+            raise RuntimeError("device timeout in the attention points")
+        out[name] = point
+        del q, k, v, o
+    return out
+
+
 def cross_roofline(B, L, H, Lk, lens, ms, peak_tflops, peak_gbs):
     """Cross-attention launch of the timed step (CUDA events around it).
     FLOPs count the true text lengths, 4 * L * len_b * 128 * H per batch row
@@ -684,11 +754,195 @@ def run_wan(args, w, rank, world, local_rank):
             n=args.hbm_elems)
     if not args.no_causal and world == 1:
         line["block_causal"] = causal_rooflines(dev, peak)
+    if not args.no_points and world == 1:
+        line["metric_points"] = attn_points(dev, pk)
     if not args.no_cpu_baseline and world == 1:
         dt, fl, text = cpu_oracle_sample(w, args.cpu_rows)
         line["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": "TFLOP/s",
                                 "cores": blas_threads(), "kind": "oracle",
                                 "sample": text, "seconds": dt}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------ Ulysses ---
+
+def ulysses_plan(L, world, rank):
+    """Sequence shard of one rank: the token count padded to a multiple of
+    the rank count (Wan2.2 source reading, ch. 8 "Ulysses"), Ls tokens per
+    rank, rank r holding tokens r * Ls .. (r + 1) * Ls - 1."""
+    from video_diffusion_transformer_self_b200 import ulysses
+    Lpad = ulysses.padded_len(L, world)
+    Ls = Lpad // world
+    return {"Lpad": Lpad, "Ls": Ls, "first": rank * Ls,
+            "end": (rank + 1) * Ls}
+
+
+def ulysses_value(B, H, L, steps, max_ms):
+    """Whole-job TFLOP/s of the sharded problem: the FLOPs of ONE full
+    self-attention (4 * B * heads * L^2 * 128) per step, over the slowest
+    rank's time -- strong scaling, the ranks split one problem."""
+    return 4.0 * B * H * L * L * 128 * steps / (max_ms / 1e3) / 1e12
+
+
+def ulysses_steps(q, k, v, g, table, rope, steps, group=None, mark=None):
+    """`steps` Ulysses self-attentions of this rank's [B, Ls, H, 128]
+    shards; mark(tag) (if given) is called with "start", "exchanged",
+    "attended" and "end" around the phases.  Returns the last output."""
+    from video_diffusion_transformer_self_b200 import ulysses
+    o = None
+    for _ in range(steps):
+        if mark:
+            mark("start")
+        o = ulysses.ulysses_self_attn(q, k, v, g, table, group=group,
+                                      rope=rope, marks=mark)
+        if mark:
+            mark("end")
+    return o
+
+
+def run_ulysses(args, w, rank, world, local_rank):
+    """One 720p-81f (or --workload) self-attention split over the ranks by
+    Ulysses: each rank holds a sequence shard of Q, K, V (all heads), three
+    all-to-alls give it the whole sequence of heads / P heads, it rotates
+    them (--rope pre) or attends with the rotation fused, and one all-to-all
+    returns its output shard.  The exchanges (pack, NCCL all-to-all,
+    unpack) and the attention are timed separately with CUDA events."""
+    import torch
+
+    from video_diffusion_transformer_self_b200 import wan
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.current_stream()
+    _, g = wan.token_grid(w.frames, w.height, w.width)
+    L, B, H = g.F * g.H * g.W, w.batch, w.heads
+    if H % world:
+        raise SystemExit("heads (%d) do not divide by %d ranks" % (H, world))
+    plan = ulysses_plan(L, world, rank)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(7070 + rank)
+    shape = (B, plan["Ls"], H, 128)
+    q, k, v = (torch.randn(shape, device=dev, generator=gen)
+               .to(torch.bfloat16) for _ in range(3))
+    table = wan.rope3d_table(g)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist_mod
+        dist = dist_mod
+
+    def barrier():
+        if dist is not None:
+            dist.barrier(device_ids=[local_rank])
+
+    events = {}
+
+    def mark(tag):
+        e = torch.cuda.Event(enable_timing=True)
+        e.record(stream)
+        events.setdefault(tag, []).append(e)
+
+    ulysses_steps(q, k, v, g, table, args.rope, args.warmup)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local_rank) if rank == 0 else None
+    barrier()
+    torch.cuda.synchronize()
+    ulysses_steps(q, k, v, g, table, args.rope, args.steps, mark=mark)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop() if clocks else None
+    if wan.device_status() != 0:
+        raise RuntimeError("device timeout during the timed steps")
+    st, ex, at, en = (events[t] for t in ("start", "exchanged", "attended",
+                                           "end"))
+    total = st[0].elapsed_time(en[-1])
+    exch = sum(a.elapsed_time(b) for a, b in zip(st, ex)) + \
+        sum(a.elapsed_time(b) for a, b in zip(at, en))
+    attn = sum(a.elapsed_time(b) for a, b in zip(ex, at))
+    total, exch, attn = max_over_ranks([total, exch, attn], dist, dev)
+
+    # end to end: every step uploads this rank's shards from pinned host
+    # memory and reads its output shard back
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+        ho = torch.empty(shape, dtype=torch.bfloat16).pin_memory()
+        dq, dk, dv = (torch.empty_like(t) for t in (q, k, v))
+
+        def e2e_steps(n):
+            for _ in range(n):
+                for d_, h_ in ((dq, hq), (dk, hk), (dv, hv)):
+                    d_.copy_(h_, non_blocking=True)
+                o = ulysses_steps(dq, dk, dv, g, table, args.rope, 1)
+                ho.copy_(o, non_blocking=True)
+
+        e2e_steps(1)
+        torch.cuda.synchronize()
+        barrier()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        e2e_steps(args.steps)
+        b.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e2e_ms = max_over_ranks([a.elapsed_time(b)], dist, dev)[0]
+        nb = 3 * q.numel() * 2
+        e2e = {"value": ulysses_value(B, H, L, args.steps, e2e_ms),
+               "unit": "TFLOP/s", "h2d_bytes_per_step": nb,
+               "d2h_bytes_per_step": q.numel() * 2,
+               "ms_per_step": e2e_ms / args.steps,
+               "pipelined": "no (copies, exchanges and kernels in order)"}
+    if rank != 0:
+        return
+    pk, pk_kind = peaks()
+    peak = float(pk.get("bf16_tflops_sustained", 1400.0))
+    value = ulysses_value(B, H, L, args.steps, total)
+    fl_rank = 4.0 * B * (H // world) * L * L * 128
+    # library launches per step: the transpose kernel packs q, k, v (and
+    # unpacks them when B > 1) and unpacks the output (packing it too when
+    # B > 1); then the RoPE pass (--rope pre) and the attention kernel
+    moves = (3 + 1 + (4 if B > 1 else 0)) if world > 1 else 0
+    per_step = moves + 1 + (1 if args.rope == "pre" else 0)
+    line = {
+        "metric": "self-attn TFLOP/s",
+        "value": value,
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": total / args.steps,
+        "higher_is_better": True,
+        "scaling": "strong",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {
+            "workload": w.name, "batch": B, "heads": H, "seq_len": L,
+            "grid": [g.F, g.H, g.W], "rope": args.rope,
+            "parallelism": "ulysses%d" % world, "tokens_per_rank":
+            plan["Ls"], "padded_tokens": plan["Lpad"],
+            "l2": "inputs larger than L2 at 720p-81f",
+        },
+        "ulysses": {
+            "exchange_ms_per_step": exch / args.steps,
+            "attention_ms_per_step": attn / args.steps,
+            "exchange_bytes_per_rank_per_step":
+                4 * B * plan["Ls"] * H * 256 * (world - 1) / world,
+            "attention_tflops_per_rank": fl_rank / (attn / args.steps / 1e3)
+                / 1e12,
+        },
+        "roofline": {
+            "kernel": "attn_fwd_kernel self-attention on heads / P",
+            "bound": "tensor",
+            "achieved": fl_rank / (attn / args.steps / 1e3) / 1e12,
+            "peak": peak, "unit": "TFLOP/s",
+            "frac": fl_rank / (attn / args.steps / 1e3) / 1e12 / peak,
+            "traffic": None, "peak_kind": pk_kind + " sustained bf16",
+        },
+        "gpu_launches": per_step * args.steps,
+        "e2e": e2e,
+        "clocks": clk,
+    }
     print(json.dumps(line), flush=True)
 
 
@@ -710,12 +964,18 @@ def main():
 
         import torch
         import torch.distributed as dist
+        if args.parallel == "ulysses":
+            # keep NCCL's communicator lines (transport, NVLS use) in the log
+            os.environ.setdefault("NCCL_DEBUG", "INFO")
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl",
                                 timeout=datetime.timedelta(seconds=120))
         dist.barrier(device_ids=[local_rank])
     try:
-        run_wan(args, w, rank, world, local_rank)
+        if args.parallel == "ulysses":
+            run_ulysses(args, w, rank, world, local_rank)
+        else:
+            run_wan(args, w, rank, world, local_rank)
     finally:
         if world > 1:
             import torch.distributed as dist

@@ -60,3 +60,52 @@ def check_guards(buf, guard):
     tail = buf[-guard:].float()
     assert torch.isnan(head).all() and torch.isnan(tail).all(), \
         "write outside the output tensor"
+
+
+def oracle_threads():
+    """Worker threads for oracle evaluations over independent heads."""
+    import os
+    try:
+        n = len(os.sched_getaffinity(0))
+    except AttributeError:
+        n = os.cpu_count() or 1
+    return max(1, min(int(os.environ.get("WAN_ORACLE_THREADS", n)), 32))
+
+
+def map_threads(fn, items):
+    """list(map(fn, items)) on a thread pool.  numpy's BLAS calls and
+    float64 ufunc loops release the GIL, so independent heads run in
+    parallel; BLAS is held to one thread per call while the pool runs (no
+    process pool: nothing is forked after the CUDA context exists)."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    from threadpoolctl import threadpool_limits
+    with threadpool_limits(limits=1, user_api="blas"):
+        with ThreadPoolExecutor(oracle_threads()) as ex:
+            return list(ex.map(fn, items))
+
+
+def head_metrics(label, got, want):
+    """(label, max-abs error, relative Frobenius error, all finite) of one
+    (batch, head) comparison."""
+    return (label, max_abs(got, want), rel_fro(got, want),
+            bool(np.all(np.isfinite(got))))
+
+
+def assert_heads_close(results, what):
+    """results: list of head_metrics(...) per (batch, head).  Every pair
+    must meet the attention tolerance; the assertion text lists the
+    max-abs and relative-Frobenius errors of every pair and the worst."""
+    worst_ma, worst_rf, lines, bad = 0.0, 0.0, [], []
+    for label, ma, rf, finite in results:
+        worst_ma, worst_rf = max(worst_ma, ma), max(worst_rf, rf)
+        ok = finite and ma <= ATTN_MAX_ABS and rf <= ATTN_REL_FRO
+        lines.append("%s max_abs %.3g rel_fro %.3g%s"
+                     % (label, ma, rf, "" if ok else "  <-- FAIL"))
+        if not ok:
+            bad.append(label)
+    assert not bad, "%s: %d of %d (b, h) over tolerance (max_abs <= %.3g, " \
+        "rel_fro <= %.3g); worst max_abs %.3g rel_fro %.3g\n%s" % (
+            what, len(bad), len(results), ATTN_MAX_ABS, ATTN_REL_FRO,
+            worst_ma, worst_rf, "\n".join(lines))
+    return worst_ma, worst_rf

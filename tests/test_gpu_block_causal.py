@@ -5,8 +5,9 @@ import numpy as np
 import pytest
 import torch
 
-from gpu_common import (assert_attn_close, check_guards, cuda, f64,
-                        guarded_empty_like, scale_for)
+from gpu_common import (assert_attn_close, assert_heads_close, check_guards,
+                        cuda, f64, guarded_empty_like, head_metrics,
+                        map_threads, scale_for)
 from oracle import attention as oattn
 from video_diffusion_transformer_self_b200 import build, inputs, wan
 
@@ -90,9 +91,11 @@ def test_480p_17f_frame_chunks():
 
 # ---- the launch configuration bench.py times: 480p-165f, 42 x 30 x 52 =
 # 65,520 tokens, 40 heads, chunks of 3 latent frames (4,680 tokens).  The
-# oracle evaluates sampled rows on a sample of heads (heads are independent).
+# oracle evaluates 4,096 seeded sampled rows of every head (heads are
+# independent and run on a thread pool), always including rows on both
+# sides of chunk boundaries.
 FULL_L, FULL_H, FULL_CHUNK = 65520, 40, 4680
-HEADS = np.array([0, 13, 27, 39])
+N_ROWS = 4096
 
 
 def _full_qkv():
@@ -100,8 +103,19 @@ def _full_qkv():
 
 
 def _rows(n_total, seed, extra=()):
-    rows = inputs.sample_rows(n_total, 96, seed).numpy()
+    rows = inputs.sample_rows(n_total, N_ROWS - len(extra), seed).numpy()
     return np.unique(np.concatenate([rows, np.asarray(extra, np.int64)]))
+
+
+def _per_head(got, q, k, v, rows, q_offset, what):
+    def one(h):
+        want = oattn.block_causal_attention(
+            f64(q[:, :, h:h + 1]), f64(k[:, :, h:h + 1]),
+            f64(v[:, :, h:h + 1]), scale_for(128), FULL_CHUNK, q_offset,
+            rows, row_block=128)
+        return head_metrics("%s h%d (%d rows)" % (what, h, len(rows)),
+                            got[:, rows, h:h + 1], want)
+    assert_heads_close(map_threads(one, range(FULL_H)), what)
 
 
 def test_full_sequence_480p_165f_sampled():
@@ -109,10 +123,7 @@ def test_full_sequence_480p_165f_sampled():
     got = _run(q, k, v, FULL_CHUNK)
     # rows on both sides of chunk boundaries and in the first chunk
     rows = _rows(FULL_L, 91, [1, 4679, 4680, 32759, 32760, 60839, 60840])
-    want = oattn.block_causal_attention(
-        f64(q[:, :, HEADS]), f64(k[:, :, HEADS]), f64(v[:, :, HEADS]),
-        scale_for(128), FULL_CHUNK, 0, rows)
-    assert_attn_close(got[:, rows][:, :, HEADS], want, "480p-165f full")
+    _per_head(got, q, k, v, rows, 0, "480p-165f full")
 
 
 def test_kv_cache_last_chunk_480p_165f_sampled():
@@ -121,7 +132,4 @@ def test_kv_cache_last_chunk_480p_165f_sampled():
     ql = q[:, q0:].contiguous()
     got = _run(ql, k, v, FULL_CHUNK, q0)
     rows = _rows(FULL_CHUNK, 92, [1, FULL_CHUNK - 2])
-    want = oattn.block_causal_attention(
-        f64(ql[:, :, HEADS]), f64(k[:, :, HEADS]), f64(v[:, :, HEADS]),
-        scale_for(128), FULL_CHUNK, q0, rows)
-    assert_attn_close(got[:, rows][:, :, HEADS], want, "480p-165f KV step")
+    _per_head(got, ql, k, v, rows, q0, "480p-165f KV step")

@@ -1,10 +1,11 @@
 """GPU parity at the full workload sizes, in the launch configuration the
 benchmark times: the whole attention call runs on the device; the oracle
-evaluates seeded sampled query rows (always including the first and last
-row, so the ragged tail tile is covered) against all keys.
+evaluates 4,096 seeded sampled query rows of every (batch row, head)
+(always including the first and last row, so the ragged tail tile is
+covered) against all keys, in fp64.
 
-Rows per (batch, head): WAN_PARITY_ROWS (default 256 at 75,600 and 65,520
-tokens, 512 at 32,760 tokens)."""
+Heads are independent, so the oracle runs them on a thread pool.  Rows per
+(batch, head): WAN_PARITY_ROWS (default 4096)."""
 
 import os
 
@@ -12,7 +13,8 @@ import numpy as np
 import pytest
 import torch
 
-from gpu_common import assert_attn_close, cuda, f64, scale_for
+from gpu_common import (assert_attn_close, assert_heads_close, cuda, f64,
+                        head_metrics, map_threads, scale_for)
 from oracle import attention as oattn
 from oracle import grid as ogrid
 from oracle import rope as orope
@@ -21,6 +23,8 @@ from video_diffusion_transformer_self_b200.workloads import WORKLOADS
 
 pytestmark = pytest.mark.gpu
 
+ROW_BLOCK = 128  # oracle rows per matmul: bounds each thread's memory
+
 
 @pytest.fixture(scope="module", autouse=True)
 def _lib():
@@ -28,8 +32,8 @@ def _lib():
     wan.lib()
 
 
-def _rows(default):
-    return int(os.environ.get("WAN_PARITY_ROWS", default))
+def _rows():
+    return int(os.environ.get("WAN_PARITY_ROWS", 4096))
 
 
 def _workload_tensors(w):
@@ -58,35 +62,43 @@ def _sampled_self_parity(widx, n_rows, mode):
     assert wan.device_status() == 0
     o = o.cpu()
     del qg, kg, vg
-    worst = (0.0, 0.0)
-    for b in range(w.batch):
-        for h in range(w.heads):
-            rows = inputs.sample_rows(
-                L, n_rows, inputs.seed_for(widx, "rows") + 1000 * b + h).numpy()
-            qh = orope.rope3d(f64(q[b:b + 1, :, h:h + 1]), grid)[:, rows]
-            kh = orope.rope3d(f64(k[b:b + 1, :, h:h + 1]), grid)
-            vh = f64(v[b:b + 1, :, h:h + 1])
-            want = oattn.attention(qh, kh, vh, scale_for())
-            got = f64(o[b:b + 1, rows, h:h + 1])
-            ma, rf = assert_attn_close(got, want, "%s b%d h%d" % (w.name, b, h))
-            worst = (max(worst[0], ma), max(worst[1], rf))
-    return worst
+    angles = orope.token_angles(grid)
+
+    def one(bh):
+        b, h = bh
+        rows = inputs.sample_rows(
+            L, n_rows, inputs.seed_for(widx, "rows") + 1000 * b + h).numpy()
+        qh = orope.apply_angles(f64(q[b:b + 1, rows, h:h + 1]), angles[rows])
+        kh = orope.apply_angles(f64(k[b:b + 1, :, h:h + 1]), angles)
+        vh = f64(v[b:b + 1, :, h:h + 1])
+        want = oattn.attention(qh, kh, vh, scale_for(), row_block=ROW_BLOCK)
+        got = f64(o[b:b + 1, rows, h:h + 1])
+        return head_metrics("%s %s b%d h%d (%d rows)"
+                            % (w.name, mode, b, h, len(rows)), got, want)
+
+    res = map_threads(one, [(b, h) for b in range(w.batch)
+                            for h in range(w.heads)])
+    return assert_heads_close(res, "%s %s" % (w.name, mode))
 
 
 def test_self_attn_480p_81f_sampled():
-    _sampled_self_parity(2, _rows(512), "fused")
+    _sampled_self_parity(2, _rows(), "fused")
+
+
+def test_self_attn_480p_81f_prerotated_sampled():
+    _sampled_self_parity(2, _rows(), "pre")
 
 
 def test_self_attn_720p_81f_sampled():
-    _sampled_self_parity(3, _rows(256), "fused")
+    _sampled_self_parity(3, _rows(), "fused")
 
 
 def test_self_attn_720p_81f_prerotated_sampled():
-    _sampled_self_parity(3, _rows(64), "pre")
+    _sampled_self_parity(3, _rows(), "pre")
 
 
 def test_self_attn_480p_165f_sampled():
-    _sampled_self_parity(4, _rows(64), "fused")
+    _sampled_self_parity(4, _rows(), "fused")
 
 
 @pytest.mark.parametrize("widx", [2, 3])
@@ -110,8 +122,18 @@ def test_cross_attn_full_size(widx):
     torch.cuda.synchronize()
     assert wan.device_status() == 0
     o = o.cpu()
-    rows = inputs.sample_rows(L, 2048, inputs.seed_for(widx, "rows")).numpy()
-    want = oattn.attention(f64(q[:, rows]), f64(kc), f64(vc), scale_for(),
-                           kv_lens=lens)
-    got = f64(o[:, rows])
-    assert_attn_close(got, want, "cross " + w.name)
+    rows = inputs.sample_rows(L, _rows(), inputs.seed_for(widx, "rows")).numpy()
+
+    def one(bh):
+        b, h = bh
+        want = oattn.attention(f64(q[b:b + 1, rows, h:h + 1]),
+                               f64(kc[b:b + 1, :, h:h + 1]),
+                               f64(vc[b:b + 1, :, h:h + 1]), scale_for(),
+                               kv_lens=[lens[b]], row_block=ROW_BLOCK)
+        got = f64(o[b:b + 1, rows, h:h + 1])
+        return head_metrics("cross %s b%d h%d len %d" % (w.name, b, h,
+                                                         lens[b]), got, want)
+
+    res = map_threads(one, [(b, h) for b in range(w.batch)
+                            for h in range(w.heads)])
+    assert_heads_close(res, "cross " + w.name)

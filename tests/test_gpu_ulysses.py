@@ -1,15 +1,18 @@
 """GPU checks of the Ulysses path: the library's block transpose against
 numpy (bit-exact), and P ranks emulated on one GPU -- every rank's pack,
 head attention and unpack run the real kernels, only the all-to-all is a
-local permutation of the send buffers -- against wan.self_attn on the whole
-sequence.  Attention heads are independent, so the sharded result must be
-bit-identical."""
+local permutation of the send buffers.  The gathered result is compared
+with the fp64 oracle on the whole, unsharded problem (at the attention
+tolerance), and with wan.self_attn on the whole sequence: attention heads
+are independent, so that must be bit-identical."""
 
 import numpy as np
 import pytest
 import torch
 
-from gpu_common import cuda
+from gpu_common import assert_attn_close, cuda, f64, scale_for
+from oracle import attention as oattn
+from oracle import rope as orope
 from video_diffusion_transformer_self_b200 import build, inputs, ulysses, wan
 
 pytestmark = pytest.mark.gpu
@@ -44,11 +47,13 @@ def _exchange(sends):
 
 
 @pytest.mark.parametrize("P,B,grid,H,rope", [
-    (2, 1, (2, 6, 10), 40, True),
-    (4, 2, (2, 6, 10), 40, True),
-    (5, 1, (2, 6, 10), 40, False),
-    (8, 1, (3, 5, 7), 40, True),     # 105 tokens padded to 112
-    (8, 1, (21, 6, 8), 8, True),     # 1,008 tokens: several key blocks
+    (2, 1, (2, 6, 10), 40, "fused"),
+    (4, 2, (2, 6, 10), 40, "fused"),
+    (5, 1, (2, 6, 10), 40, None),
+    (8, 1, (3, 5, 7), 40, "fused"),  # 105 tokens padded to 112
+    (8, 1, (21, 6, 8), 8, "fused"),  # 1,008 tokens: several key blocks
+    (4, 1, (21, 6, 8), 8, "pre"),    # rotation after the exchange
+    (8, 1, (3, 5, 7), 40, "pre"),    # ... with padding
 ])
 def test_emulated_ranks_equal_unsharded(P, B, grid, H, rope):
     g = wan.grid(*grid)
@@ -60,7 +65,12 @@ def test_emulated_ranks_equal_unsharded(P, B, grid, H, rope):
             for r in ("q", "k", "v")]
     table = wan.rope3d_table(g) if rope else None
     want = torch.empty((B, L, H, 128), dtype=torch.bfloat16, device="cuda")
-    wan.self_attn(*[cuda(t[:, :L]) for t in full], want, g, table=table)
+    qw, kw, vw = [cuda(t[:, :L]) for t in full]
+    if rope == "pre":
+        wan.rope3d_qk(qw, kw, g, table)
+        wan.self_attn(qw, kw, vw, want, g)
+    else:
+        wan.self_attn(qw, kw, vw, want, g, table=table)
     # rank r holds tokens r * Ls .. (r + 1) * Ls - 1 of every tensor
     shards = [[cuda(t[:, r * Ls:(r + 1) * Ls]) for t in full]
               for r in range(P)]
@@ -71,11 +81,19 @@ def test_emulated_ranks_equal_unsharded(P, B, grid, H, rope):
         heads.append([ulysses.unpack_seq_to_head(recv)
                       for recv in _exchange(sends)])
     outs_h = [ulysses.head_attention(heads[0][r], heads[1][r], heads[2][r],
-                                     g, table) for r in range(P)]
+                                     g, table, rope=rope or "fused")
+              for r in range(P)]
     sends = [ulysses.pack_head_to_seq(oh, P) for oh in outs_h]
     outs = [ulysses.unpack_head_to_seq(recv) for recv in _exchange(sends)]
     torch.cuda.synchronize()
     assert wan.device_status() == 0
     got = torch.cat(outs, dim=1)[:, :L]
     assert got.shape == want.shape
+    # the fp64 oracle on the whole, unsharded problem
+    qd, kd, vd = (f64(t[:, :L]) for t in full)
+    if rope:
+        qd, kd = orope.rope3d(qd, grid), orope.rope3d(kd, grid)
+    assert_attn_close(f64(got), oattn.attention(qd, kd, vd, scale_for()),
+                      "Ulysses P=%d B=%d %s" % (P, B, rope))
+    # and bit-identical to the unsharded kernel: heads are independent
     assert torch.equal(got, want)

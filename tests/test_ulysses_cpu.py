@@ -37,6 +37,8 @@ def _cpu_swap(inp, out, a, b, row_bytes):
 
 def _oracle_attention(q, k, v, o, g, table, scale):
     assert table is None
+    if scale is None:  # the library's default, 1 / sqrt(head_dim)
+        scale = 1 / math.sqrt(q.shape[-1])
     o.copy_(torch.from_numpy(oattn.attention(
         q.double().numpy(), k.double().numpy(), v.double().numpy(),
         scale)).to(o.dtype))
@@ -131,3 +133,58 @@ def test_rejects_bad_splits():
         ulysses.pack_seq_to_head(torch.zeros(1, 2, 6, 128), 4)  # 6 % 4
     with pytest.raises(ValueError):
         ulysses.pack_head_to_seq(torch.zeros(1, 6, 2, 128), 4)  # 6 % 4
+
+
+# ---- bench.py --parallel ulysses: its host logic on two gloo ranks, with
+# the same CPU stand-ins for the two kernels.
+
+def _bench_worker(rank, world, port, out):
+    import bench
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    ulysses._swap = _cpu_swap
+    ulysses._attention = _oracle_attention
+    try:
+        grid, B, H = (3, 3, 3), 1, 4          # 27 tokens -> 28 on 2 ranks
+        L = 27
+        plan = bench.ulysses_plan(L, world, rank)
+        q, k, v = _full_inputs(B, plan["Lpad"], H, 5)
+        sl = slice(plan["first"], plan["end"])
+        tags = []
+        o = bench.ulysses_steps(q[:, sl].contiguous(), k[:, sl].contiguous(),
+                                v[:, sl].contiguous(), wan.grid(*grid), None,
+                                "pre", 2, mark=tags.append)
+        red = bench.max_over_ranks([1.0 + rank, 5.0 - rank], dist, "cpu")
+        out[rank] = (plan, o.clone(), tags, red)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_bench_ulysses_mode_two_gloo_ranks():
+    import bench
+    world = 2
+    with mp.get_context("spawn").Manager() as m:
+        out = m.dict()
+        mp.spawn(_bench_worker, args=(world, _free_port(), out),
+                 nprocs=world, join=True)
+        res = dict(out)
+    plans = [res[r][0] for r in range(world)]
+    # equal shards covering the padded sequence, in rank order
+    assert [p["Ls"] for p in plans] == [14, 14]
+    assert plans[0]["first"] == 0 and plans[1]["first"] == 14
+    assert plans[1]["end"] == plans[0]["Lpad"] == 28
+    # phases marked in order, once per step
+    assert res[0][2] == ["start", "exchanged", "attended", "end"] * 2
+    # timings reduce to the slowest rank
+    assert res[0][3] == res[1][3] == [2.0, 5.0]
+    q, k, v = _full_inputs(1, 28, 4, 5)
+    want = oattn.attention(q[:, :27].double().numpy(),
+                           k[:, :27].double().numpy(),
+                           v[:, :27].double().numpy(), 1 / math.sqrt(128))
+    got = torch.cat([res[r][1] for r in range(world)], dim=1)[:, :27]
+    np.testing.assert_allclose(got.double().numpy(), want, rtol=0,
+                               atol=2e-6 * np.abs(want).max())
+    # strong scaling: one problem's FLOPs, not one per rank
+    assert bench.ulysses_value(1, 40, 75600, 10, 1000.0) == pytest.approx(
+        4.0 * 40 * 75600 ** 2 * 128 * 10 / 1e12)

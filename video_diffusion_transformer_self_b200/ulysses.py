@@ -40,6 +40,10 @@ def _attention(q, k, v, o, g, table, softmax_scale):
     wan.self_attn(q, k, v, o, g, table=table, softmax_scale=softmax_scale)
 
 
+def _rope(q, k, g, table):
+    wan.rope3d_qk(q, k, g, table)
+
+
 def _world(group):
     return dist.get_world_size(group) if dist.is_initialized() else 1
 
@@ -116,29 +120,42 @@ def head_to_seq(y, group=None):
 
 # ------------------------------------------------------------ attention --
 
-def head_attention(qh, kh, vh, g, table=None, softmax_scale=None):
+def head_attention(qh, kh, vh, g, table=None, softmax_scale=None,
+                   rope="fused"):
     """Attention of head-sharded [B, Lpad, Hp, d] tensors over the grid g's
-    L = F * H * W tokens; rows past L (padding) are left unspecified."""
+    L = F * H * W tokens; rows past L (padding) are left unspecified.
+
+    With a table, rope="fused" rotates q and k inside the attention kernel's
+    tile stage; rope="pre" first rotates the received q and k in place with
+    the stand-alone RoPE pass (each holds the whole sequence of its heads,
+    so every token's (f, h, w) is known) and then attends without a table.
+    """
+    if rope not in ("fused", "pre"):
+        raise ValueError("rope must be 'fused' or 'pre'")
     B, Lpad = qh.shape[0], qh.shape[1]
     L = g.F * g.H * g.W
     oh = torch.empty_like(qh)
-    if Lpad == L:
-        _attention(qh, kh, vh, oh, g, table, softmax_scale)
-    else:
-        if B != 1:
-            raise ValueError("sequence padding needs batch 1")
-        _attention(qh[:, :L], kh[:, :L], vh[:, :L], oh[:, :L], g, table,
-                   softmax_scale)
+    if Lpad != L and B != 1:
+        raise ValueError("sequence padding needs batch 1")
+    q_, k_, v_, o_ = ((qh, kh, vh, oh) if Lpad == L else
+                      (qh[:, :L], kh[:, :L], vh[:, :L], oh[:, :L]))
+    if table is not None and rope == "pre":
+        _rope(q_, k_, g, table)
+        table = None
+    _attention(q_, k_, v_, o_, g, table, softmax_scale)
     return oh
 
 
 def ulysses_self_attn(q, k, v, g, table=None, softmax_scale=None,
-                      group=None):
+                      group=None, rope="fused", marks=None):
     """Self-attention over the token grid g from sequence shards.
 
     q, k, v: [B, Ls, H, 128] bf16 on this rank's GPU, rank r holding tokens
     r * Ls .. (r + 1) * Ls - 1 of the sequence padded to P * Ls =
     padded_len(F * H * W, P).  Returns this rank's [B, Ls, H, 128] output.
+    rope: see head_attention.  marks: optional callable, called with
+    "exchanged" after the three inbound exchanges and with "attended" after
+    the attention (used to time the two phases).
     """
     P = _world(group)
     L = g.F * g.H * g.W
@@ -149,5 +166,9 @@ def ulysses_self_attn(q, k, v, g, table=None, softmax_scale=None,
     qh = seq_to_head(q, group)
     kh = seq_to_head(k, group)
     vh = seq_to_head(v, group)
-    oh = head_attention(qh, kh, vh, g, table, softmax_scale)
+    if marks is not None:
+        marks("exchanged")
+    oh = head_attention(qh, kh, vh, g, table, softmax_scale, rope)
+    if marks is not None:
+        marks("attended")
     return head_to_seq(oh, group)
