@@ -115,6 +115,17 @@ int wan_self_attn(const void* q, const void* k, const void* v, void* o,
                   int B, wan_grid_t g, int heads, int head_dim,
                   const void* d_table, float softmax_scale, void* s);
 
+/* The same full self-attention (q and k already rotated) computed by pairs
+ * of CTAs on two SMs: one tcgen05 MMA (cta_group::2) covers 256 query rows,
+ * 128 in each SM's tensor memory, with each SM staging half of every K / V
+ * block; three score slots per SM let the Q K^T of later blocks run while
+ * the softmax of an earlier one is still going.  Same layouts, arguments,
+ * errors and results as wan_self_attn with d_table == NULL.  Source: Wan2.2
+ * source reading, ch. 4 "Full forward of one block" and ch. 8.            */
+int wan_self_attn_pair(const void* q, const void* k, const void* v, void* o,
+                       int B, wan_grid_t g, int heads, int head_dim,
+                       float softmax_scale, void* s);
+
 /* ------------------------------------------------------ cross-attention --
  * Wan2.2 source reading, ch. 3 "Where did the prompt go" (each prompt is
  * trimmed to its true length; video tokens query, the text context is

@@ -768,6 +768,402 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ============================================================ CTA pairs ==
+//
+// Self-attention over pairs of CTAs on two SMs.  One tcgen05 MMA with
+// cta_group::2 multiplies a 256-row query tile (128 rows in each CTA's
+// tensor memory) by a 128-key block whose K rows (for Q K^T) and V channels
+// (for P V) are split between the two CTAs' shared memory, so each SM
+// stages half of every K / V block and the B operand costs each SM half the
+// shared-memory bandwidth.  That frees tensor memory for a ring of three
+// score slots per CTA: S(j+1) and S(j+2) are computed while the softmax of
+// block j runs, and the softmax of one block never waits on the P V and
+// Q K^T of the previous one (the two-tile kernel above has that chain).
+//
+// Per CTA (320 threads):
+//   warps 0-7  softmax: warp w owns query rows 32 (w & 3) .. + 31 (TMEM
+//              lane quadrant w & 3) and keys 64 (w >> 2) .. + 63 of every
+//              block; the two warps of a quadrant swap row maxima through
+//              shared memory (an mbarrier per quadrant), rescale their half
+//              of O when the max grows by more than 2^8, and write P (bf16)
+//              over the scores they have read.
+//   warp 8     TMA producer: this CTA's Q rows, its 64 keys of each K block
+//              (3 blocks ahead of V) and its 64 channels of each V block.
+//   warp 9     in CTA 0: the MMA issuer for the pair; in CTA 1: forwards the
+//              completion of CTA 1's loads to CTA 0 (remote mbarrier arrive).
+// Tensor memory (512 columns, both CTAs): O at 0, score slot b at 128 + 128 b;
+// P of keys 0-63 / 64-127 over score columns 0-31 / 64-95 of the slot.
+namespace pair {
+constexpr int RM = 128;                    // query rows per CTA
+constexpr int NSLOT = 3;                   // score / P slots
+constexpr int PNSK = 5;                     // K stages (64 keys each)
+constexpr int PNSV = 4;                     // V stages (64 channels each)
+constexpr uint32_t QHALF = 16384;          // [128 rows][64 ch] bf16
+constexpr uint32_t QTILE = 2 * QHALF;
+constexpr uint32_t KHALF = 8192;           // [64 keys][64 ch] bf16
+constexpr uint32_t KTILE = 2 * KHALF;
+constexpr uint32_t VTILE = 16384;          // [128 keys][64 ch] bf16
+constexpr uint32_t SMEM = QTILE + PNSK * KTILE + PNSV * VTILE + 1024;
+constexpr int THREADS = 320;
+constexpr uint32_t TM_SLOT0 = 128;
+constexpr uint16_t BOTH = 3;               // multicast mask: CTAs 0 and 1
+constexpr uint32_t IDESC_S2 = idesc_bf16_f32(2 * RM, BN, 0);
+constexpr uint32_t IDESC_PV2 = idesc_bf16_f32(2 * RM, HD, 1);
+
+enum : int {
+  QFULL = 0,                  // this CTA's Q landed (local)
+  QPEER = 1,                  // CTA 1's Q landed (CTA 0 only)
+  KFULL = 2,                  // per K stage, local
+  KPEER = KFULL + PNSK,        // per K stage, CTA 1's half landed (CTA 0)
+  VFULL = KPEER + PNSK,
+  VPEER = VFULL + PNSV,
+  KEMPTY = VPEER + PNSV,       // per stage: the pair's MMAs are done with it
+  VEMPTY = KEMPTY + PNSK,
+  SFULL = VEMPTY + PNSV,       // per slot: S written (both CTAs)
+  PREADY = SFULL + NSLOT,     // per slot: P written by all 16 softmax warps
+  PVDONE = PREADY + NSLOT,    // per slot: P V done (both CTAs)
+  OFINAL = PVDONE + NSLOT,    // the item's last P V done (both CTAs)
+  DRAIN = OFINAL + 1,         // every MMA done (both CTAs)
+  XCH = DRAIN + 1,            // per lane quadrant: both key halves posted
+  PNBAR = XCH + 4
+};
+}  // namespace pair
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::THREADS, 1)
+    attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
+                     const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_v,
+                     const __grid_constant__ AttnArgs args) {
+  using namespace pair;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t bar[PNBAR];
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_abort;
+  __shared__ float s_xch[2][2][RM];  // [block parity][key half][row]
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool lead = rank == 0;
+  volatile int* abort_flag = &s_abort;
+  int* status = &g_wan_status;
+
+  // Same offsets in both CTAs: the MMAs address both with one descriptor.
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* sm = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  uint8_t* sQ = sm;
+  uint8_t* sK = sm + QTILE;
+  uint8_t* sV = sK + PNSK * KTILE;
+
+  const int item = static_cast<int>(blockIdx.x >> 1);
+  const int tx = item % args.n_tiles_x;
+  const int head = (item / args.n_tiles_x) % args.heads;
+  const int bb = item / args.n_tiles_x / args.heads;
+  const int q0 = tx * (2 * RM) + static_cast<int>(rank) * RM;
+  const int kv_len = args.Lk;
+  const int nblk = (kv_len + BN - 1) / BN;
+
+  if (threadIdx.x == 0) {
+    s_abort = 0;
+    mbar_init(&bar[QFULL], 1);
+    mbar_init(&bar[QPEER], 1);
+    for (int i = 0; i < PNSK; ++i) {
+      mbar_init(&bar[KFULL + i], 1);
+      mbar_init(&bar[KPEER + i], 1);
+      mbar_init(&bar[KEMPTY + i], 1);
+    }
+    for (int i = 0; i < PNSV; ++i) {
+      mbar_init(&bar[VFULL + i], 1);
+      mbar_init(&bar[VPEER + i], 1);
+      mbar_init(&bar[VEMPTY + i], 1);
+    }
+    for (int i = 0; i < NSLOT; ++i) {
+      mbar_init(&bar[SFULL + i], 1);
+      mbar_init(&bar[PREADY + i], 16);
+      mbar_init(&bar[PVDONE + i], 1);
+    }
+    mbar_init(&bar[OFINAL], 1);
+    mbar_init(&bar[DRAIN], 1);
+    for (int i = 0; i < 4; ++i) mbar_init(&bar[XCH + i], 2);
+    fence_mbar_init();
+  }
+  if (warp == 9) tmem_alloc_pair(&s_tmem, 512);
+  tc_fence_before();
+  __syncthreads();
+  // the peer's barriers are initialised before any remote arrive or commit
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+
+  if (warp == 8) {
+    // --------------------------------------------------------- producer --
+    const bool el = elect_one();
+    if (el) {
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      mbar_expect_tx(&bar[QFULL], QTILE);
+      tma_load_4d(sQ, &tm_q, &bar[QFULL], 0, head, q0, bb);
+      tma_load_4d(sQ + QHALF, &tm_q, &bar[QFULL], 64, head, q0, bb);
+    }
+    __syncwarp();
+    bool ok = true;
+    int nk = 0, nv = 0;
+    // K of block j goes out with V of block j - NSLOT: the order the MMA
+    // warp consumes them (S runs NSLOT blocks ahead of P V).
+    for (int j = 0; j < nblk + NSLOT && ok; ++j) {
+      if (j < nblk) {
+        const int sk = j % PNSK;
+        if (j >= PNSK)
+          ok = wait_warp_cl(&bar[KEMPTY + sk], ((j / PNSK) - 1) & 1,
+                            abort_flag, status);
+        if (!ok) break;
+        if (el) {
+          const int key0 = j * BN + static_cast<int>(rank) * 64;
+          mbar_expect_tx(&bar[KFULL + sk], KTILE);
+          tma_load_4d(sK + sk * KTILE, &tm_k, &bar[KFULL + sk], 0, head, key0,
+                      bb);
+          tma_load_4d(sK + sk * KTILE + KHALF, &tm_k, &bar[KFULL + sk], 64,
+                      head, key0, bb);
+        }
+        __syncwarp();
+        ++nk;
+      }
+      const int jv = j - NSLOT;
+      if (jv >= 0) {
+        const int sv = jv % PNSV;
+        if (jv >= PNSV)
+          ok = wait_warp_cl(&bar[VEMPTY + sv], ((jv / PNSV) - 1) & 1,
+                            abort_flag, status);
+        if (!ok) break;
+        if (el) {
+          mbar_expect_tx(&bar[VFULL + sv], VTILE);
+          tma_load_4d(sV + sv * VTILE, &tm_v, &bar[VFULL + sv],
+                      static_cast<int>(rank) * 64, head, jv * BN, bb);
+        }
+        __syncwarp();
+        ++nv;
+      }
+    }
+    if (*abort_flag) {
+      // copies already issued land in this CTA before it leaves
+      wait_warp_drain(&bar[QFULL], 0, status);
+      for (int g = (nk > PNSK ? nk - PNSK : 0); g < nk; ++g)
+        wait_warp_drain(&bar[KFULL + g % PNSK], (g / PNSK) & 1, status);
+      for (int g = (nv > PNSV ? nv - PNSV : 0); g < nv; ++g)
+        wait_warp_drain(&bar[VFULL + g % PNSV], (g / PNSV) & 1, status);
+    }
+  } else if (warp == 9 && !lead) {
+    // ----------------------------------- CTA 1: forward load completions --
+    auto fwd = [&](int full, int peer, uint32_t parity) -> bool {
+      if (!wait_warp_cl(&bar[full], parity, abort_flag, status)) return false;
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&bar[peer]), 0));
+      __syncwarp();
+      return true;
+    };
+    bool ok = fwd(QFULL, QPEER, 0);
+    for (int j = 0; j < nblk + NSLOT && ok; ++j) {
+      if (j < nblk)
+        ok = fwd(KFULL + j % PNSK, KPEER + j % PNSK, (j / PNSK) & 1);
+      const int jv = j - NSLOT;
+      if (ok && jv >= 0)
+        ok = fwd(VFULL + jv % PNSV, VPEER + jv % PNSV, (jv / PNSV) & 1);
+    }
+    // every MMA of the pair is done before this CTA's memory is released
+    wait_warp_cl_drain(&bar[DRAIN], 0, status);
+  } else if (warp == 9) {
+    // ---------------------------------------------- CTA 0: MMA issuer --
+    const uint64_t dq = sdesc_sw128(smem_u32(sQ), 16, 1024);
+    const uint64_t dk = sdesc_sw128(smem_u32(sK), 16, 1024);
+    // V: MN-major, one 64-channel swizzle atom per CTA, 8-key groups 1 KB
+    const uint64_t dv = sdesc_sw128(smem_u32(sV), 16, 1024);
+    const bool el = elect_one();
+    bool ok = wait_warp_cl(&bar[QFULL], 0, abort_flag, status) &&
+              wait_warp_cl(&bar[QPEER], 0, abort_flag, status);
+    // S(j) = Q K(j)^T into slot j % NSLOT of both CTAs.
+    auto issue_s = [&](int j) -> bool {
+      const int sk = j % PNSK;
+      const uint32_t ph = (j / PNSK) & 1;
+      if (!wait_warp_cl(&bar[KFULL + sk], ph, abort_flag, status) ||
+          !wait_warp_cl(&bar[KPEER + sk], ph, abort_flag, status))
+        return false;
+      tc_fence_after();
+      const uint64_t b0 = dk + ((sk * KTILE) >> 4);
+      const uint32_t d = tmem + TM_SLOT0 + (j % NSLOT) * 128;
+      if (el) {
+#pragma unroll
+        for (int k = 0; k < HD / 16; ++k) {
+          const uint32_t oa = ((k >> 2) * QHALF + (k & 3) * 32) >> 4;
+          const uint32_t ob = ((k >> 2) * KHALF + (k & 3) * 32) >> 4;
+          umma_ss_pair(d, dq + oa, b0 + ob, IDESC_S2, k > 0 ? 1u : 0u);
+        }
+        umma_commit_pair(&bar[SFULL + j % NSLOT], BOTH);
+        umma_commit_pair(&bar[KEMPTY + sk], BOTH);
+      }
+      __syncwarp();
+      return true;
+    };
+    for (int j = 0; j < NSLOT && j < nblk && ok; ++j) ok = issue_s(j);
+    for (int j = 0; j < nblk && ok; ++j) {
+      const int sl = j % NSLOT, sv = j % PNSV;
+      const uint32_t pv = (j / PNSV) & 1;
+      ok = wait_warp_cl(&bar[PREADY + sl], (j / NSLOT) & 1, abort_flag,
+                        status) &&
+           wait_warp_cl(&bar[VFULL + sv], pv, abort_flag, status) &&
+           wait_warp_cl(&bar[VPEER + sv], pv, abort_flag, status);
+      if (!ok) break;
+      tc_fence_after();
+      const uint64_t b0 = dv + ((sv * VTILE) >> 4);
+      const uint32_t a0 = tmem + TM_SLOT0 + sl * 128;
+      if (el) {
+#pragma unroll
+        for (int k = 0; k < BN / 16; ++k) {
+          // P of keys 16k .. 16k+15: key half k >> 2 at column 64 (k >> 2)
+          umma_ts_pair(tmem, a0 + 64 * (k >> 2) + 8 * (k & 3),
+                       b0 + ((k * 2048) >> 4), IDESC_PV2,
+                       (j > 0 || k > 0) ? 1u : 0u);
+        }
+        umma_commit_pair(&bar[PVDONE + sl], BOTH);
+        umma_commit_pair(&bar[VEMPTY + sv], BOTH);
+      }
+      __syncwarp();
+      // the slot's P is consumed (MMAs run in issue order): S(j + NSLOT)
+      if (j + NSLOT < nblk) ok = issue_s(j + NSLOT);
+    }
+    if (ok && el) umma_commit_pair(&bar[OFINAL], BOTH);
+    if (el) umma_commit_pair(&bar[DRAIN], BOTH);
+    __syncwarp();
+    wait_warp_cl_drain(&bar[DRAIN], 0, status);
+  } else if (warp < 8) {
+    // ---------------------------------------------------------- softmax --
+    const int qd = warp & 3;
+    const int h = warp >> 2;
+    const int r = qd * 32 + lane;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(qd * 32) << 16);
+    const uint32_t o_col = lane_base + 64 * h;
+    const float c2 = args.scale_log2;
+    float m_run = -INFINITY;
+    float l_run = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nblk && ok; ++j) {
+      const int sl = j % NSLOT;
+      ok = wait_warp_cl(&bar[SFULL + sl], (j / NSLOT) & 1, abort_flag,
+                        status);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t s_col = lane_base + TM_SLOT0 + sl * 128 + 64 * h;
+      float s[64];
+      tmem_ld64(s_col, s);
+      tmem_ld_wait64(s);
+      const int lim = kv_len - j * BN - 64 * h;  // valid keys of this half
+      const bool masked = __any_sync(0xffffffffu, lim < 64);
+      if (masked) {
+#pragma unroll
+        for (int c = 0; c < 64; ++c)
+          if (c >= lim) s[c] = -INFINITY;
+      }
+      float mx = (masked ? rowmax_masked<64>(s) : rowmax<64>(s)) * c2;
+      // both key halves of the row: swap maxima with the quadrant's partner
+      s_xch[j & 1][h][r] = mx;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar[XCH + qd]);
+      ok = wait_warp(&bar[XCH + qd], j & 1, abort_flag, status);
+      if (!ok) break;
+      mx = fmaxf(mx, s_xch[j & 1][h ^ 1][r]);
+      if (j == 0) {
+        m_run = mx;
+      } else {
+        // Keep the running max unless it grew by more than 2^8 (p <= 256,
+        // exact after the final O / l); otherwise rescale this warp's half
+        // of O once P V(j-1) has landed in it.  Both warps of the quadrant
+        // see the same maxima, so they take the same decision.
+        const bool need = mx > m_run + RESCALE_LOG2;
+        if (__any_sync(0xffffffffu, need)) {
+          const float m_new = need ? mx : m_run;
+          const float alpha = ex2(m_run - m_new);
+          ok = wait_warp_cl(&bar[PVDONE + (j - 1) % NSLOT],
+                            ((j - 1) / NSLOT) & 1, abort_flag, status);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            float o[32];
+            tmem_ld32(o_col + c * 32, o);
+            tmem_ld_wait32(o);
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              const float2 v =
+                  ffma2(make_float2(o[e], o[e + 1]),
+                        make_float2(alpha, alpha), make_float2(0.f, 0.f));
+              o[e] = v.x;
+              o[e + 1] = v.y;
+            }
+            tmem_st32(o_col + c * 32, o);
+          }
+          l_run *= alpha;
+          m_run = m_new;
+        }
+      }
+      float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                       make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+      if (masked)
+        exp_store_chunks<false>(s, c2, m_run, s_col, acc, 0, 2);
+      else
+        exp_store_chunks<true>(s, c2, m_run, s_col, acc, 0, 2);
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0)
+        mbar_arrive_cluster(mapa_shared(smem_u32(&bar[PREADY + sl]), 0));
+      const float2 tsum = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
+      l_run += tsum.x + tsum.y;
+    }
+    if (ok) ok = wait_warp_cl(&bar[OFINAL], 0, abort_flag, status);
+    if (ok) {
+      // row sum over both key halves
+      s_xch[nblk & 1][h][r] = l_run;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar[XCH + qd]);
+      ok = wait_warp(&bar[XCH + qd], nblk & 1, abort_flag, status);
+    }
+    if (ok) {
+      tc_fence_after();
+      const float inv = 1.0f / (l_run + s_xch[nblk & 1][h ^ 1][r]);
+      const int row = q0 + r;
+      __nv_bfloat16* orow =
+          args.o + ((static_cast<int64_t>(bb) * args.Lq + row) * args.heads +
+                    head) * HD + 64 * h;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        float o[32];
+        tmem_ld32(o_col + c * 32, o);
+        tmem_ld_wait32(o);
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          pk[e] = pack_bf16x2(o[2 * e] * inv, o[2 * e + 1] * inv);
+        if (row < args.Lq) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2],
+                                pk[4 * e + 3]);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  // neither CTA frees its memory while the pair's MMAs or the peer's
+  // arrivals may still reach it
+  cluster_sync_all();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, 512);
+  }
+}
+
 // One warp waits, with the same bounded wait the attention kernel uses, on
 // an mbarrier that needs one arrival and receives `arrive` (0 or 1).  With
 // none the wait runs out after kWaitLimitNs, records WAN_ETIMEOUT in the
@@ -789,51 +1185,6 @@ __global__ void __launch_bounds__(32) wait_selftest_kernel(int arrive) {
 }
 
 // ------------------------------------------------------------------ host --
-
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType,
-                                  cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion,
-                                  CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static std::once_flag once;
-  static EncodeTiledFn fn = nullptr;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000,
-                                         cudaEnableDefault,
-                                         &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  });
-  return fn;
-}
-
-// Tensor map of a [B, L, heads, 128] bf16 tensor with a [1][128][1][64] box
-// (128 tokens x 64 channels of one head), 128-byte swizzle, zero fill past L.
-int make_map(CUtensorMap* m, const void* base, int B, int L, int heads) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return WAN_ECUDA;
-  cuuint64_t dims[4] = {static_cast<cuuint64_t>(HD),
-                        static_cast<cuuint64_t>(heads),
-                        static_cast<cuuint64_t>(L),
-                        static_cast<cuuint64_t>(B)};
-  // byte strides of dims 1..3 (heads, L, B)
-  const cuuint64_t row = static_cast<cuuint64_t>(heads) * HD * 2;
-  cuuint64_t strides[3] = {static_cast<cuuint64_t>(HD) * 2, row,
-                           row * static_cast<cuuint64_t>(L)};
-  cuuint32_t box[4] = {64, 1, BM, 1};
-  cuuint32_t estr[4] = {1, 1, 1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
-                  const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? WAN_OK : WAN_EINVAL;
-}
 
 template <int kRope, int kPersist>
 int launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
@@ -887,6 +1238,32 @@ int launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
   return cudaGetLastError() == cudaSuccess ? WAN_OK : WAN_ECUDA;
 }
 
+int launch_pair(const CUtensorMap& mq, const CUtensorMap& mk,
+                const CUtensorMap& mv, AttnArgs a, int B, cudaStream_t s) {
+  static std::mutex mu;
+  static int state[64];  // 0 unknown, 1 ready
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+    return WAN_ECUDA;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (state[dev] == 0) {
+      if (cudaFuncSetAttribute(attn_pair_kernel,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               pair::SMEM) != cudaSuccess)
+        return WAN_ECUDA;
+      state[dev] = 1;
+    }
+  }
+  a.n_tiles_x = (a.Lq + 2 * pair::RM - 1) / (2 * pair::RM);
+  const int64_t items = static_cast<int64_t>(a.n_tiles_x) * a.heads * B;
+  if (2 * items > INT32_MAX) return WAN_EINVAL;
+  a.items = static_cast<int>(items);
+  attn_pair_kernel<<<static_cast<unsigned>(2 * items), pair::THREADS,
+                     pair::SMEM, s>>>(mq, mk, mv, a);
+  return cudaGetLastError() == cudaSuccess ? WAN_OK : WAN_ECUDA;
+}
+
 int check_common(const void* q, const void* k, const void* v, void* o, int B,
                  int Lq, int Lk, int heads, int head_dim,
                  float softmax_scale) {
@@ -924,9 +1301,9 @@ int wan_self_attn(const void* q, const void* k, const void* v, void* o,
   st = check_device(nullptr);
   if (st != WAN_OK) return st;
   CUtensorMap mq, mk, mv;
-  if ((st = make_map(&mq, q, B, L, heads)) != WAN_OK) return st;
-  if ((st = make_map(&mk, k, B, L, heads)) != WAN_OK) return st;
-  if ((st = make_map(&mv, v, B, L, heads)) != WAN_OK) return st;
+  if ((st = make_map_bf16(&mq, q, B, L, heads, BM)) != WAN_OK) return st;
+  if ((st = make_map_bf16(&mk, k, B, L, heads, BM)) != WAN_OK) return st;
+  if ((st = make_map_bf16(&mv, v, B, L, heads, BM)) != WAN_OK) return st;
   AttnArgs a;
   a.o = static_cast<__nv_bfloat16*>(o);
   a.table = static_cast<const float4*>(d_table);
@@ -944,6 +1321,38 @@ int wan_self_attn(const void* q, const void* k, const void* v, void* o,
                  : launch<0, 0>(mq, mk, mv, a, B, as_stream(s));
 }
 
+int wan_self_attn_pair(const void* q, const void* k, const void* v, void* o,
+                       int B, wan_grid_t g, int heads, int head_dim,
+                       float softmax_scale, void* s) {
+  using namespace wan;
+  if (g.F < 1 || g.H < 1 || g.W < 1) return WAN_EINVAL;
+  const int64_t L64 = static_cast<int64_t>(g.F) * g.H * g.W;
+  if (L64 > (1 << 26)) return WAN_EINVAL;
+  const int L = static_cast<int>(L64);
+  int st = check_common(q, k, v, o, B, L, L, heads, head_dim, softmax_scale);
+  if (st != WAN_OK) return st;
+  st = check_device(nullptr);
+  if (st != WAN_OK) return st;
+  CUtensorMap mq, mk, mv;
+  if ((st = make_map_bf16(&mq, q, B, L, heads, 128)) != WAN_OK) return st;
+  if ((st = make_map_bf16(&mk, k, B, L, heads, 64)) != WAN_OK) return st;
+  if ((st = make_map_bf16(&mv, v, B, L, heads, 128)) != WAN_OK) return st;
+  AttnArgs a;
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.table = nullptr;
+  a.Lq = L;
+  a.Lk = L;
+  a.heads = heads;
+  a.F = g.F;
+  a.H = g.H;
+  a.W = g.W;
+  a.scale_log2 = softmax_scale * 1.4426950408889634f;
+  a.cross = 0;
+  a.chunk = 0;
+  a.q_offset = 0;
+  return launch_pair(mq, mk, mv, a, B, as_stream(s));
+}
+
 int wan_block_causal_attn(const void* q, const void* k, const void* v,
                           void* o, int B, int Lq, int Lk, int heads,
                           int head_dim, int chunk_tokens, int q_offset,
@@ -958,9 +1367,9 @@ int wan_block_causal_attn(const void* q, const void* k, const void* v,
   st = check_device(nullptr);
   if (st != WAN_OK) return st;
   CUtensorMap mq, mk, mv;
-  if ((st = make_map(&mq, q, B, Lq, heads)) != WAN_OK) return st;
-  if ((st = make_map(&mk, k, B, Lk, heads)) != WAN_OK) return st;
-  if ((st = make_map(&mv, v, B, Lk, heads)) != WAN_OK) return st;
+  if ((st = make_map_bf16(&mq, q, B, Lq, heads, BM)) != WAN_OK) return st;
+  if ((st = make_map_bf16(&mk, k, B, Lk, heads, BM)) != WAN_OK) return st;
+  if ((st = make_map_bf16(&mv, v, B, Lk, heads, BM)) != WAN_OK) return st;
   AttnArgs a;
   a.o = static_cast<__nv_bfloat16*>(o);
   a.table = nullptr;
@@ -988,9 +1397,9 @@ int wan_cross_attn(const void* q, const void* k_ctx, const void* v_ctx,
   st = check_device(nullptr);
   if (st != WAN_OK) return st;
   CUtensorMap mq, mk, mv;
-  if ((st = make_map(&mq, q, B, Lq, heads)) != WAN_OK) return st;
-  if ((st = make_map(&mk, k_ctx, B, Lk, heads)) != WAN_OK) return st;
-  if ((st = make_map(&mv, v_ctx, B, Lk, heads)) != WAN_OK) return st;
+  if ((st = make_map_bf16(&mq, q, B, Lq, heads, BM)) != WAN_OK) return st;
+  if ((st = make_map_bf16(&mk, k_ctx, B, Lk, heads, BM)) != WAN_OK) return st;
+  if ((st = make_map_bf16(&mv, v_ctx, B, Lk, heads, BM)) != WAN_OK) return st;
   AttnArgs a;
   a.o = static_cast<__nv_bfloat16*>(o);
   a.table = nullptr;

@@ -27,6 +27,56 @@ int check_device(int* device_out) {
   return cached[dev] == 1 ? WAN_OK : WAN_EUNSUPPORTED;
 }
 
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType,
+                                  cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000,
+                                         cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+}  // namespace
+
+int make_map_bf16(CUtensorMap* m, const void* base, int B, int L, int heads,
+                  int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return WAN_ECUDA;
+  if (box_rows < 1 || box_rows > 256) return WAN_EINVAL;
+  constexpr int HD = 128;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(HD),
+                        static_cast<cuuint64_t>(heads),
+                        static_cast<cuuint64_t>(L),
+                        static_cast<cuuint64_t>(B)};
+  // byte strides of dims 1..3 (heads, L, B)
+  const cuuint64_t row = static_cast<cuuint64_t>(heads) * HD * 2;
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(HD) * 2, row,
+                           row * static_cast<cuuint64_t>(L)};
+  cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(box_rows), 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+                  const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? WAN_OK : WAN_EINVAL;
+}
+
 }  // namespace wan
 
 extern "C" {

@@ -19,6 +19,12 @@ namespace wan {
 // else WAN_EUNSUPPORTED / WAN_ECUDA.  Result cached per device.
 int check_device(int* device_out);
 
+// Tensor map of a [B, L, heads, 128] bf16 tensor with a box of box_rows
+// tokens x 64 channels of one head (dims: channel, head, token, batch),
+// 128-byte swizzle, zero fill past L.
+int make_map_bf16(CUtensorMap* m, const void* base, int B, int L, int heads,
+                  int box_rows);
+
 inline bool aligned16(const void* p) {
   return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
 }
@@ -424,6 +430,234 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
 
 __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// ------------------------------------------------- CTA pairs (clusters) --
+// Used by the kernels that run one MMA over a pair of CTAs on two SMs
+// (tcgen05 cta_group::2).  Every tcgen05 alloc / mma / commit in such a
+// kernel uses cta_group::2; loads and stores of tensor memory have no group.
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// All threads of both CTAs: release this CTA's prior writes, wait for the
+// peer (cluster-wide barrier).
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+               "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Address of the same shared-memory object in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr,
+                                                uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;"
+               : "=r"(r)
+               : "r"(saddr), "r"(rank));
+  return r;
+}
+
+// Arrive (release at cluster scope) on an mbarrier given by its
+// shared::cluster address (this CTA's or the peer's).
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile(
+      "mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(
+          cluster_addr)
+      : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar,
+                                                      uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;"
+      "\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// wait_warp with cluster-scope acquire: for barriers that receive arrivals
+// from the peer CTA or commits of MMAs that read the peer's memory.
+__device__ __forceinline__ bool wait_warp_cl(uint64_t* bar, uint32_t parity,
+                                             volatile int* abort_flag,
+                                             int* status) {
+  const uint32_t a = smem_u32(bar);
+  const int lane = threadIdx.x & 31;
+  if (__all_sync(0xffffffffu, mbar_try_wait_cluster(a, parity))) return true;
+  uint64_t t0 = 0;
+  for (uint32_t it = 0;; ++it) {
+    bool done = mbar_try_wait_cluster(a, parity);
+    if (__any_sync(0xffffffffu, done)) {
+      if (!done) done = mbar_try_wait_cluster(a, parity);
+      if (__all_sync(0xffffffffu, done)) return true;
+    }
+    if ((it & 31u) == 31u) {
+      int bad = 0;
+      if (lane == 0) {
+        if (*abort_flag) {
+          bad = 1;
+        } else {
+          const uint64_t now = globaltimer_ns();
+          if (t0 == 0) {
+            t0 = now;
+          } else if (now - t0 > kWaitLimitNs) {
+            bad = 1;
+            *abort_flag = 1;
+            atomicExch(status, WAN_ETIMEOUT);
+          }
+        }
+      }
+      if (__shfl_sync(0xffffffffu, bad, 0)) return false;
+    }
+  }
+}
+
+// Drain form of wait_warp_cl (ignores the abort flag, still bounded).
+__device__ __forceinline__ bool wait_warp_cl_drain(uint64_t* bar,
+                                                   uint32_t parity,
+                                                   int* status) {
+  const uint32_t a = smem_u32(bar);
+  const int lane = threadIdx.x & 31;
+  uint64_t t0 = 0;
+  for (uint32_t it = 0;; ++it) {
+    bool done = mbar_try_wait_cluster(a, parity);
+    if (__any_sync(0xffffffffu, done)) {
+      if (!done) done = mbar_try_wait_cluster(a, parity);
+      if (__all_sync(0xffffffffu, done)) return true;
+    }
+    if ((it & 31u) == 31u) {
+      int bad = 0;
+      if (lane == 0) {
+        const uint64_t now = globaltimer_ns();
+        if (t0 == 0) {
+          t0 = now;
+        } else if (now - t0 > kWaitLimitNs) {
+          bad = 1;
+          atomicExch(status, WAN_ETIMEOUT);
+        }
+      }
+      if (__shfl_sync(0xffffffffu, bad, 0)) return false;
+    }
+  }
+}
+
+// Tensor memory for a CTA pair: one warp of each CTA (same warp index)
+// allocates / frees; both CTAs get the same base address.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst,
+                                                uint32_t ncols) {
+  asm volatile(
+      "tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::
+          "r"(smem_u32(dst)),
+      "r"(ncols)
+      : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::
+                   : "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr,
+                                                  uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(
+                   taddr),
+               "r"(ncols)
+               : "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T over the CTA pair: M = 256 rows, 128 in
+// each CTA's tensor memory; A from each CTA's own shared memory (its 128
+// rows), B split by N between the two CTAs (same offsets in both).
+__device__ __forceinline__ void umma_ss_pair(uint32_t d_tmem, uint64_t a_desc,
+                                             uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Same with A from each CTA's tensor memory.
+__device__ __forceinline__ void umma_ts_pair(uint32_t d_tmem, uint32_t a_tmem,
+                                             uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(
+          d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrive on the mbarrier at this shared offset in every CTA of `mask` when
+// all pair MMAs issued so far by this thread are done.
+__device__ __forceinline__ void umma_commit_pair(uint64_t* bar,
+                                                 uint16_t mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster."
+      "multicast::cluster.b64 [%0], %1;" ::"r"(smem_u32(bar)),
+      "h"(mask)
+      : "memory");
+}
+
+// 32 lanes x 64 columns of 32-bit TMEM -> 64 registers per thread.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float* v) {
+  uint32_t* r = reinterpret_cast<uint32_t*>(v);
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 {"
+      "%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, "
+      "%24, %25, %26, %27, %28, %29, %30, %31, %32, %33, %34, %35, "
+      "%36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, "
+      "%48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, "
+      "%60, %61, %62, %63}, [%64];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]),
+        "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]),
+        "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]),
+        "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]),
+        "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]),
+        "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]),
+        "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]),
+        "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]),
+        "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]),
+        "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_ld_wait64(float* v) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+f"(v[0]), "+f"(v[1]), "+f"(v[2]), "+f"(v[3]), "+f"(v[4]),
+                 "+f"(v[5]), "+f"(v[6]), "+f"(v[7]), "+f"(v[8]), "+f"(v[9]),
+                 "+f"(v[10]), "+f"(v[11]), "+f"(v[12]), "+f"(v[13]),
+                 "+f"(v[14]), "+f"(v[15]), "+f"(v[16]), "+f"(v[17]),
+                 "+f"(v[18]), "+f"(v[19]), "+f"(v[20]), "+f"(v[21]),
+                 "+f"(v[22]), "+f"(v[23]), "+f"(v[24]), "+f"(v[25]),
+                 "+f"(v[26]), "+f"(v[27]), "+f"(v[28]), "+f"(v[29]),
+                 "+f"(v[30]), "+f"(v[31]), "+f"(v[32]), "+f"(v[33]),
+                 "+f"(v[34]), "+f"(v[35]), "+f"(v[36]), "+f"(v[37]),
+                 "+f"(v[38]), "+f"(v[39]), "+f"(v[40]), "+f"(v[41]),
+                 "+f"(v[42]), "+f"(v[43]), "+f"(v[44]), "+f"(v[45]),
+                 "+f"(v[46]), "+f"(v[47]), "+f"(v[48]), "+f"(v[49]),
+                 "+f"(v[50]), "+f"(v[51]), "+f"(v[52]), "+f"(v[53]),
+                 "+f"(v[54]), "+f"(v[55]), "+f"(v[56]), "+f"(v[57]),
+                 "+f"(v[58]), "+f"(v[59]), "+f"(v[60]), "+f"(v[61]),
+                 "+f"(v[62]), "+f"(v[63])::"memory");
+}
+
+// Named barrier over `nthreads` threads (a multiple of 32).
+__device__ __forceinline__ void named_bar_sync(uint32_t id,
+                                               uint32_t nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 // Hardware base-2 exponential (MUFU), flush-to-zero.

@@ -67,6 +67,8 @@ _SIGNATURES = {
     "wan_rope3d_qk": (_I, [_P, _P, _I, Grid, _I, _I, _P, _P]),
     "wan_self_attn": (_I, [_P, _P, _P, _P, _I, Grid, _I, _I, _P,
                            ctypes.c_float, _P]),
+    "wan_self_attn_pair": (_I, [_P, _P, _P, _P, _I, Grid, _I, _I,
+                                ctypes.c_float, _P]),
     "wan_cross_attn": (_I, [_P, _P, _P, _P, ctypes.POINTER(ctypes.c_int32),
                             _I, _I, _I, _I, _I, ctypes.c_float, _P]),
     "wan_block_causal_attn": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I,
@@ -270,6 +272,24 @@ def self_attn(q, k, v, o, g, table=None, softmax_scale=None, stream=None):
     _check(lib().wan_self_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, g, H, D,
                                _ptr(table), softmax_scale, _stream(stream)),
            "wan_self_attn")
+
+
+def self_attn_pair(q, k, v, o, g, softmax_scale=None, stream=None):
+    """o = softmax(q k^T * scale) v over the grid's tokens (q, k already
+    rotated), computed by the CTA-pair kernel (one MMA over two SMs)."""
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o)):
+        _bf16_bl(t, name)
+        _shape_is(t, q.shape, name)
+    B, L, H, D = q.shape
+    if L != _grid_tokens(g):
+        raise ValueError("q holds %d tokens, grid %r has %d"
+                         % (L, g, _grid_tokens(g)))
+    _on_cuda(("q", q), ("k", k), ("v", v), ("o", o))
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(D)
+    _check(lib().wan_self_attn_pair(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, g,
+                                    H, D, softmax_scale, _stream(stream)),
+           "wan_self_attn_pair")
 
 
 def cross_attn(q, k_ctx, v_ctx, o, ctx_lens, softmax_scale=None,
