@@ -160,6 +160,15 @@ int wan_block_causal_attn(const void* q, const void* k, const void* v,
                           int head_dim, int chunk_tokens, int q_offset,
                           float softmax_scale, void* s);
 
+/* The same block-causal attention computed by pairs of CTAs on two SMs (the
+ * kernel of wan_self_attn_pair, with the per-row key limit above; the
+ * 256-row tiles of each head run heaviest first).  Same arguments, layouts,
+ * errors and results as wan_block_causal_attn.                            */
+int wan_block_causal_attn_pair(const void* q, const void* k, const void* v,
+                               void* o, int B, int Lq, int Lk, int heads,
+                               int head_dim, int chunk_tokens, int q_offset,
+                               float softmax_scale, void* s);
+
 /* ---------------------------------------- block prologue and epilogue --
  * Wan2.2 source reading, ch. 4, section "Full forward of one block": the
  * self-attention input is norm1(x) * (1 + e[1]) + e[0] and the block output

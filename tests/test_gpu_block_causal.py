@@ -20,10 +20,10 @@ def _lib():
     wan.lib()
 
 
-def _run(q, k, v, chunk, q_offset=0):
+def _run(q, k, v, chunk, q_offset=0, pair=False):
     qg, kg, vg = cuda(q), cuda(k), cuda(v)
     o, buf, guard = guarded_empty_like(qg)
-    wan.block_causal_attn(qg, kg, vg, o, chunk, q_offset)
+    wan.block_causal_attn(qg, kg, vg, o, chunk, q_offset, pair=pair)
     torch.cuda.synchronize()
     assert wan.device_status() == 0
     check_guards(buf, guard)
@@ -37,6 +37,7 @@ def _qkv(B, Lq, Lk, H, seed):
     return q, k, v
 
 
+@pytest.mark.parametrize("pair", [False, True], ids=["tiles", "pair"])
 @pytest.mark.parametrize("B,L,H,chunk", [
     (1, 300, 2, 50),     # chunks inside tiles, several per CTA
     (2, 700, 1, 128),    # chunk = one key block
@@ -45,45 +46,48 @@ def _qkv(B, Lq, Lk, H, seed):
     (1, 333, 2, 333),    # one chunk = full attention
     (1, 1000, 1, 2000),  # chunk longer than the sequence
 ])
-def test_full_sequence(B, L, H, chunk):
+def test_full_sequence(B, L, H, chunk, pair):
     q, k, v = _qkv(B, L, L, H, 500 + L)
-    got = _run(q, k, v, chunk)
+    got = _run(q, k, v, chunk, pair=pair)
     want = oattn.block_causal_attention(f64(q), f64(k), f64(v), scale_for(),
                                         chunk)
     assert_attn_close(got, want, "block-causal L=%d chunk=%d" % (L, chunk))
 
 
+@pytest.mark.parametrize("pair", [False, True], ids=["tiles", "pair"])
 @pytest.mark.parametrize("chunk,n_chunks", [(120, 5), (1560, 3)])
-def test_kv_cache_chunk_step(chunk, n_chunks):
+def test_kv_cache_chunk_step(chunk, n_chunks, pair):
     # the last chunk's queries against the cached prefix + itself
     L = chunk * n_chunks
     q, k, v = _qkv(1, L, L, 2, 900 + chunk)
     off = L - chunk
-    got = _run(q[:, off:].contiguous(), k, v, chunk, q_offset=off)
+    got = _run(q[:, off:].contiguous(), k, v, chunk, q_offset=off, pair=pair)
     want = oattn.block_causal_attention(f64(q[:, off:]), f64(k), f64(v),
                                         scale_for(), chunk, q_offset=off)
     assert_attn_close(got, want, "kv-cache chunk %d" % chunk)
 
 
-def test_first_chunk_ignores_later_keys():
+@pytest.mark.parametrize("pair", [False, True], ids=["tiles", "pair"])
+def test_first_chunk_ignores_later_keys(pair):
     chunk, L = 96, 400
     q, k, v = _qkv(1, L, L, 1, 77)
     k2 = (k.float() + 5.0).to(torch.bfloat16)
     v2 = (v.float() - 3.0).to(torch.bfloat16)
     k2[:, :chunk] = k[:, :chunk]
     v2[:, :chunk] = v[:, :chunk]
-    a = _run(q[:, :chunk].contiguous(), k, v, chunk)
-    b = _run(q[:, :chunk].contiguous(), k2, v2, chunk)
+    a = _run(q[:, :chunk].contiguous(), k, v, chunk, pair=pair)
+    b = _run(q[:, :chunk].contiguous(), k2, v2, chunk, pair=pair)
     # keys past the first chunk get weight exactly 0 (they may share a
     # loaded key block with visible keys): changing them changes no bit
     assert np.array_equal(a, b)
 
 
-def test_480p_17f_frame_chunks():
+@pytest.mark.parametrize("pair", [False, True], ids=["tiles", "pair"])
+def test_480p_17f_frame_chunks(pair):
     # 7,800 tokens, chunk = one latent frame (1,560 tokens), 12 heads
     L, H, chunk = 7800, 12, 1560
     q, k, v = _qkv(1, L, L, H, inputs.seed_for(1, "q"))
-    got = _run(q, k, v, chunk)
+    got = _run(q, k, v, chunk, pair=pair)
     want = oattn.block_causal_attention(f64(q), f64(k), f64(v), scale_for(),
                                         chunk)
     assert_attn_close(got, want, "block-causal 7800")
@@ -118,18 +122,20 @@ def _per_head(got, q, k, v, rows, q_offset, what):
     assert_heads_close(map_threads(one, range(FULL_H)), what)
 
 
-def test_full_sequence_480p_165f_sampled():
+@pytest.mark.parametrize("pair", [False, True], ids=["tiles", "pair"])
+def test_full_sequence_480p_165f_sampled(pair):
     q, k, v = _full_qkv()
-    got = _run(q, k, v, FULL_CHUNK)
+    got = _run(q, k, v, FULL_CHUNK, pair=pair)
     # rows on both sides of chunk boundaries and in the first chunk
     rows = _rows(FULL_L, 91, [1, 4679, 4680, 32759, 32760, 60839, 60840])
     _per_head(got, q, k, v, rows, 0, "480p-165f full")
 
 
-def test_kv_cache_last_chunk_480p_165f_sampled():
+@pytest.mark.parametrize("pair", [False, True], ids=["tiles", "pair"])
+def test_kv_cache_last_chunk_480p_165f_sampled(pair):
     q, k, v = _full_qkv()
     q0 = FULL_L - FULL_CHUNK
     ql = q[:, q0:].contiguous()
-    got = _run(ql, k, v, FULL_CHUNK, q0)
+    got = _run(ql, k, v, FULL_CHUNK, q0, pair=pair)
     rows = _rows(FULL_CHUNK, 92, [1, FULL_CHUNK - 2])
     _per_head(got, ql, k, v, rows, q0, "480p-165f KV step")

@@ -791,20 +791,23 @@ __global__ void __launch_bounds__(kThreads, 1)
 //              (3 blocks ahead of V) and its 64 channels of each V block.
 //   warp 9     in CTA 0: the MMA issuer for the pair; in CTA 1: forwards the
 //              completion of CTA 1's loads to CTA 0 (remote mbarrier arrive).
+//   warps 10-11  (kRopeQ) rotate this CTA's 128 query rows by the 3D RoPE
+//              once, in shared memory, before any MMA reads them; K comes
+//              in already rotated.
 // Tensor memory (512 columns, both CTAs): O at 0, score slot b at 128 + 128 b;
 // P of keys 0-63 / 64-127 over score columns 0-31 / 64-95 of the slot.
 namespace pair {
 constexpr int RM = 128;                    // query rows per CTA
 constexpr int NSLOT = 3;                   // score / P slots
-constexpr int PNSK = 5;                     // K stages (64 keys each)
-constexpr int PNSV = 4;                     // V stages (64 channels each)
+constexpr int KSTAGES = 5;                     // K stages (64 keys each)
+constexpr int VSTAGES = 4;                     // V stages (64 channels each)
 constexpr uint32_t QHALF = 16384;          // [128 rows][64 ch] bf16
 constexpr uint32_t QTILE = 2 * QHALF;
 constexpr uint32_t KHALF = 8192;           // [64 keys][64 ch] bf16
 constexpr uint32_t KTILE = 2 * KHALF;
 constexpr uint32_t VTILE = 16384;          // [128 keys][64 ch] bf16
-constexpr uint32_t SMEM = QTILE + PNSK * KTILE + PNSV * VTILE + 1024;
-constexpr int THREADS = 320;
+constexpr uint32_t SMEM = QTILE + KSTAGES * KTILE + VSTAGES * VTILE + 1024;
+constexpr int THREADS = 320;               // 384 with the Q-rotation warps
 constexpr uint32_t TM_SLOT0 = 128;
 constexpr uint16_t BOTH = 3;               // multicast mask: CTAs 0 and 1
 constexpr uint32_t IDESC_S2 = idesc_bf16_f32(2 * RM, BN, 0);
@@ -814,29 +817,32 @@ enum : int {
   QFULL = 0,                  // this CTA's Q landed (local)
   QPEER = 1,                  // CTA 1's Q landed (CTA 0 only)
   KFULL = 2,                  // per K stage, local
-  KPEER = KFULL + PNSK,        // per K stage, CTA 1's half landed (CTA 0)
-  VFULL = KPEER + PNSK,
-  VPEER = VFULL + PNSV,
-  KEMPTY = VPEER + PNSV,       // per stage: the pair's MMAs are done with it
-  VEMPTY = KEMPTY + PNSK,
-  SFULL = VEMPTY + PNSV,       // per slot: S written (both CTAs)
+  KPEER = KFULL + KSTAGES,        // per K stage, CTA 1's half landed (CTA 0)
+  VFULL = KPEER + KSTAGES,
+  VPEER = VFULL + VSTAGES,
+  KEMPTY = VPEER + VSTAGES,       // per stage: the pair's MMAs are done with it
+  VEMPTY = KEMPTY + KSTAGES,
+  SFULL = VEMPTY + VSTAGES,       // per slot: S written (both CTAs)
   PREADY = SFULL + NSLOT,     // per slot: P written by all 16 softmax warps
   PVDONE = PREADY + NSLOT,    // per slot: P V done (both CTAs)
   OFINAL = PVDONE + NSLOT,    // the item's last P V done (both CTAs)
   DRAIN = OFINAL + 1,         // every MMA done (both CTAs)
   XCH = DRAIN + 1,            // per lane quadrant: both key halves posted
-  PNBAR = XCH + 4
+  QREADY = XCH + 4,           // (kRopeQ) this CTA's Q rows rotated
+  NUM_BARS = QREADY + 1
 };
 }  // namespace pair
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::THREADS, 1)
+template <int kRopeQ>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(
+    pair::THREADS + 64 * kRopeQ, 1)
     attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v,
                      const __grid_constant__ AttnArgs args) {
   using namespace pair;
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t bar[PNBAR];
+  __shared__ __align__(8) uint64_t bar[NUM_BARS];
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
   __shared__ float s_xch[2][2][RM];  // [block parity][key half][row]
@@ -853,26 +859,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::THREADS, 1)
   uint8_t* sm = smem_raw + (((raw + 1023u) & ~1023u) - raw);
   uint8_t* sQ = sm;
   uint8_t* sK = sm + QTILE;
-  uint8_t* sV = sK + PNSK * KTILE;
+  uint8_t* sV = sK + KSTAGES * KTILE;
 
+  // Work item of the pair: 256 query rows of one (head, batch row); the
+  // block-causal mode runs the tiles of a head heaviest first.
   const int item = static_cast<int>(blockIdx.x >> 1);
   const int tx = item % args.n_tiles_x;
   const int head = (item / args.n_tiles_x) % args.heads;
   const int bb = item / args.n_tiles_x / args.heads;
-  const int q0 = tx * (2 * RM) + static_cast<int>(rank) * RM;
-  const int kv_len = args.Lk;
+  const int tile = args.chunk ? args.n_tiles_x - 1 - tx : tx;
+  const int q0 = tile * (2 * RM) + static_cast<int>(rank) * RM;
+  int kv_len = args.Lk;
+  if (args.chunk) {
+    // keys visible to the pair's last query row (both CTAs agree)
+    const int last = min(tile * (2 * RM) + 2 * RM, args.Lq) - 1 + args.q_offset;
+    kv_len = min(args.Lk, (last / args.chunk + 1) * args.chunk);
+  }
   const int nblk = (kv_len + BN - 1) / BN;
 
   if (threadIdx.x == 0) {
     s_abort = 0;
     mbar_init(&bar[QFULL], 1);
     mbar_init(&bar[QPEER], 1);
-    for (int i = 0; i < PNSK; ++i) {
+    for (int i = 0; i < KSTAGES; ++i) {
       mbar_init(&bar[KFULL + i], 1);
       mbar_init(&bar[KPEER + i], 1);
       mbar_init(&bar[KEMPTY + i], 1);
     }
-    for (int i = 0; i < PNSV; ++i) {
+    for (int i = 0; i < VSTAGES; ++i) {
       mbar_init(&bar[VFULL + i], 1);
       mbar_init(&bar[VPEER + i], 1);
       mbar_init(&bar[VEMPTY + i], 1);
@@ -885,6 +899,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::THREADS, 1)
     mbar_init(&bar[OFINAL], 1);
     mbar_init(&bar[DRAIN], 1);
     for (int i = 0; i < 4; ++i) mbar_init(&bar[XCH + i], 2);
+    mbar_init(&bar[QREADY], 64);
     fence_mbar_init();
   }
   if (warp == 9) tmem_alloc_pair(&s_tmem, 512);
@@ -913,9 +928,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::THREADS, 1)
     // warp consumes them (S runs NSLOT blocks ahead of P V).
     for (int j = 0; j < nblk + NSLOT && ok; ++j) {
       if (j < nblk) {
-        const int sk = j % PNSK;
-        if (j >= PNSK)
-          ok = wait_warp_cl(&bar[KEMPTY + sk], ((j / PNSK) - 1) & 1,
+        const int sk = j % KSTAGES;
+        if (j >= KSTAGES)
+          ok = wait_warp_cl(&bar[KEMPTY + sk], ((j / KSTAGES) - 1) & 1,
                             abort_flag, status);
         if (!ok) break;
         if (el) {
@@ -931,9 +946,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::THREADS, 1)
       }
       const int jv = j - NSLOT;
       if (jv >= 0) {
-        const int sv = jv % PNSV;
-        if (jv >= PNSV)
-          ok = wait_warp_cl(&bar[VEMPTY + sv], ((jv / PNSV) - 1) & 1,
+        const int sv = jv % VSTAGES;
+        if (jv >= VSTAGES)
+          ok = wait_warp_cl(&bar[VEMPTY + sv], ((jv / VSTAGES) - 1) & 1,
                             abort_flag, status);
         if (!ok) break;
         if (el) {
@@ -948,10 +963,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::THREADS, 1)
     if (*abort_flag) {
       // copies already issued land in this CTA before it leaves
       wait_warp_drain(&bar[QFULL], 0, status);
-      for (int g = (nk > PNSK ? nk - PNSK : 0); g < nk; ++g)
-        wait_warp_drain(&bar[KFULL + g % PNSK], (g / PNSK) & 1, status);
-      for (int g = (nv > PNSV ? nv - PNSV : 0); g < nv; ++g)
-        wait_warp_drain(&bar[VFULL + g % PNSV], (g / PNSV) & 1, status);
+      for (int g = (nk > KSTAGES ? nk - KSTAGES : 0); g < nk; ++g)
+        wait_warp_drain(&bar[KFULL + g % KSTAGES], (g / KSTAGES) & 1, status);
+      for (int g = (nv > VSTAGES ? nv - VSTAGES : 0); g < nv; ++g)
+        wait_warp_drain(&bar[VFULL + g % VSTAGES], (g / VSTAGES) & 1, status);
     }
   } else if (warp == 9 && !lead) {
     // ----------------------------------- CTA 1: forward load completions --
@@ -961,13 +976,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::THREADS, 1)
       __syncwarp();
       return true;
     };
-    bool ok = fwd(QFULL, QPEER, 0);
+    bool ok = fwd(kRopeQ ? QREADY : QFULL, QPEER, 0);
     for (int j = 0; j < nblk + NSLOT && ok; ++j) {
       if (j < nblk)
-        ok = fwd(KFULL + j % PNSK, KPEER + j % PNSK, (j / PNSK) & 1);
+        ok = fwd(KFULL + j % KSTAGES, KPEER + j % KSTAGES, (j / KSTAGES) & 1);
       const int jv = j - NSLOT;
       if (ok && jv >= 0)
-        ok = fwd(VFULL + jv % PNSV, VPEER + jv % PNSV, (jv / PNSV) & 1);
+        ok = fwd(VFULL + jv % VSTAGES, VPEER + jv % VSTAGES, (jv / VSTAGES) & 1);
     }
     // every MMA of the pair is done before this CTA's memory is released
     wait_warp_cl_drain(&bar[DRAIN], 0, status);
@@ -978,12 +993,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::THREADS, 1)
     // V: MN-major, one 64-channel swizzle atom per CTA, 8-key groups 1 KB
     const uint64_t dv = sdesc_sw128(smem_u32(sV), 16, 1024);
     const bool el = elect_one();
-    bool ok = wait_warp_cl(&bar[QFULL], 0, abort_flag, status) &&
-              wait_warp_cl(&bar[QPEER], 0, abort_flag, status);
+    bool ok =
+        wait_warp_cl(&bar[kRopeQ ? QREADY : QFULL], 0, abort_flag, status) &&
+        wait_warp_cl(&bar[QPEER], 0, abort_flag, status);
     // S(j) = Q K(j)^T into slot j % NSLOT of both CTAs.
     auto issue_s = [&](int j) -> bool {
-      const int sk = j % PNSK;
-      const uint32_t ph = (j / PNSK) & 1;
+      const int sk = j % KSTAGES;
+      const uint32_t ph = (j / KSTAGES) & 1;
       if (!wait_warp_cl(&bar[KFULL + sk], ph, abort_flag, status) ||
           !wait_warp_cl(&bar[KPEER + sk], ph, abort_flag, status))
         return false;
@@ -1005,8 +1021,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::THREADS, 1)
     };
     for (int j = 0; j < NSLOT && j < nblk && ok; ++j) ok = issue_s(j);
     for (int j = 0; j < nblk && ok; ++j) {
-      const int sl = j % NSLOT, sv = j % PNSV;
-      const uint32_t pv = (j / PNSV) & 1;
+      const int sl = j % NSLOT, sv = j % VSTAGES;
+      const uint32_t pv = (j / VSTAGES) & 1;
       ok = wait_warp_cl(&bar[PREADY + sl], (j / NSLOT) & 1, abort_flag,
                         status) &&
            wait_warp_cl(&bar[VFULL + sv], pv, abort_flag, status) &&
@@ -1034,6 +1050,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::THREADS, 1)
     if (el) umma_commit_pair(&bar[DRAIN], BOTH);
     __syncwarp();
     wait_warp_cl_drain(&bar[DRAIN], 0, status);
+  } else if (kRopeQ && warp >= 10) {
+    // ------------------------------------------------ Q rotation (RoPE) --
+    const int tr = threadIdx.x - 320;  // 0..63
+    if (wait_warp_cl(&bar[QFULL], 0, abort_flag, status)) {
+      for (int rr = tr; rr < RM; rr += 64)
+        if (q0 + rr < args.Lq) rope_row(sQ, rr, q0 + rr, args);
+      fence_proxy_async_smem();
+      mbar_arrive(&bar[QREADY]);
+    }
   } else if (warp < 8) {
     // ---------------------------------------------------------- softmax --
     const int qd = warp & 3;
@@ -1042,6 +1067,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::THREADS, 1)
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(qd * 32) << 16);
     const uint32_t o_col = lane_base + 64 * h;
     const float c2 = args.scale_log2;
+    // keys this row may see: all kv_len, or its block-causal limit
+    int row_lim = kv_len;
+    if (args.chunk && q0 + r < args.Lq) {
+      const int pos = q0 + r + args.q_offset;
+      row_lim = min(args.Lk, (pos / args.chunk + 1) * args.chunk);
+    }
     float m_run = -INFINITY;
     float l_run = 0.f;
     bool ok = true;
@@ -1055,7 +1086,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::THREADS, 1)
       float s[64];
       tmem_ld64(s_col, s);
       tmem_ld_wait64(s);
-      const int lim = kv_len - j * BN - 64 * h;  // valid keys of this half
+      const int lim = row_lim - j * BN - 64 * h;  // valid keys of this half
       const bool masked = __any_sync(0xffffffffu, lim < 64);
       if (masked) {
 #pragma unroll
@@ -1238,6 +1269,7 @@ int launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
   return cudaGetLastError() == cudaSuccess ? WAN_OK : WAN_ECUDA;
 }
 
+template <int kRopeQ>
 int launch_pair(const CUtensorMap& mq, const CUtensorMap& mk,
                 const CUtensorMap& mv, AttnArgs a, int B, cudaStream_t s) {
   static std::mutex mu;
@@ -1248,7 +1280,7 @@ int launch_pair(const CUtensorMap& mq, const CUtensorMap& mk,
   {
     std::lock_guard<std::mutex> lock(mu);
     if (state[dev] == 0) {
-      if (cudaFuncSetAttribute(attn_pair_kernel,
+      if (cudaFuncSetAttribute(attn_pair_kernel<kRopeQ>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                pair::SMEM) != cudaSuccess)
         return WAN_ECUDA;
@@ -1259,8 +1291,9 @@ int launch_pair(const CUtensorMap& mq, const CUtensorMap& mk,
   const int64_t items = static_cast<int64_t>(a.n_tiles_x) * a.heads * B;
   if (2 * items > INT32_MAX) return WAN_EINVAL;
   a.items = static_cast<int>(items);
-  attn_pair_kernel<<<static_cast<unsigned>(2 * items), pair::THREADS,
-                     pair::SMEM, s>>>(mq, mk, mv, a);
+  attn_pair_kernel<kRopeQ>
+      <<<static_cast<unsigned>(2 * items), pair::THREADS + 64 * kRopeQ,
+         pair::SMEM, s>>>(mq, mk, mv, a);
   return cudaGetLastError() == cudaSuccess ? WAN_OK : WAN_ECUDA;
 }
 
@@ -1350,7 +1383,38 @@ int wan_self_attn_pair(const void* q, const void* k, const void* v, void* o,
   a.cross = 0;
   a.chunk = 0;
   a.q_offset = 0;
-  return launch_pair(mq, mk, mv, a, B, as_stream(s));
+  return launch_pair<0>(mq, mk, mv, a, B, as_stream(s));
+}
+
+int wan_block_causal_attn_pair(const void* q, const void* k, const void* v,
+                               void* o, int B, int Lq, int Lk, int heads,
+                               int head_dim, int chunk_tokens, int q_offset,
+                               float softmax_scale, void* s) {
+  using namespace wan;
+  int st = check_common(q, k, v, o, B, Lq, Lk, heads, head_dim,
+                        softmax_scale);
+  if (st != WAN_OK) return st;
+  if (chunk_tokens < 1 || q_offset < 0 ||
+      static_cast<int64_t>(q_offset) + Lq > Lk)
+    return WAN_EINVAL;
+  st = check_device(nullptr);
+  if (st != WAN_OK) return st;
+  CUtensorMap mq, mk, mv;
+  if ((st = make_map_bf16(&mq, q, B, Lq, heads, 128)) != WAN_OK) return st;
+  if ((st = make_map_bf16(&mk, k, B, Lk, heads, 64)) != WAN_OK) return st;
+  if ((st = make_map_bf16(&mv, v, B, Lk, heads, 128)) != WAN_OK) return st;
+  AttnArgs a;
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.table = nullptr;
+  a.Lq = Lq;
+  a.Lk = Lk;
+  a.heads = heads;
+  a.F = a.H = a.W = 1;
+  a.scale_log2 = softmax_scale * 1.4426950408889634f;
+  a.cross = 0;
+  a.chunk = chunk_tokens;
+  a.q_offset = q_offset;
+  return launch_pair<0>(mq, mk, mv, a, B, as_stream(s));
 }
 
 int wan_block_causal_attn(const void* q, const void* k, const void* v,

@@ -73,6 +73,8 @@ _SIGNATURES = {
                             _I, _I, _I, _I, _I, ctypes.c_float, _P]),
     "wan_block_causal_attn": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I,
                                    _I, ctypes.c_float, _P]),
+    "wan_block_causal_attn_pair": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I,
+                                        _I, _I, ctypes.c_float, _P]),
     "wan_adaln_modulate": (_I, [_P, _P, _P, _P, _I, _I, _I, ctypes.c_float,
                                 _P]),
     "wan_qk_norm_rope": (_I, [_P, _P, _P, _P, _I, Grid, _I, _I, _P,
@@ -315,9 +317,10 @@ def cross_attn(q, k_ctx, v_ctx, o, ctx_lens, softmax_scale=None,
 
 
 def block_causal_attn(q, k, v, o, chunk_tokens, q_offset=0,
-                      softmax_scale=None, stream=None):
+                      softmax_scale=None, stream=None, pair=False):
     """Chunk-wise causal attention: query a = q_offset + i sees keys
-    j < (a // chunk_tokens + 1) * chunk_tokens (and j < Lk)."""
+    j < (a // chunk_tokens + 1) * chunk_tokens (and j < Lk).  pair=True runs
+    the CTA-pair kernel (wan_block_causal_attn_pair)."""
     for name, t in (("q", q), ("k", k), ("v", v), ("o", o)):
         _bf16_bl(t, name)
     B, Lq, H, D = q.shape
@@ -328,11 +331,11 @@ def block_causal_attn(q, k, v, o, chunk_tokens, q_offset=0,
     _on_cuda(("q", q), ("k", k), ("v", v), ("o", o))
     if softmax_scale is None:
         softmax_scale = 1.0 / math.sqrt(D)
-    _check(lib().wan_block_causal_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(o),
-                                       B, Lq, Lk, H, D, int(chunk_tokens),
-                                       int(q_offset), softmax_scale,
-                                       _stream(stream)),
-           "wan_block_causal_attn")
+    fn = lib().wan_block_causal_attn_pair if pair else \
+        lib().wan_block_causal_attn
+    _check(fn(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, Lq, Lk, H, D,
+              int(chunk_tokens), int(q_offset), softmax_scale,
+              _stream(stream)), "wan_block_causal_attn")
 
 
 def _f32(t, name):
