@@ -39,7 +39,14 @@ def parse():
     p.add_argument("--steps", type=int, default=10)
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--workload", default="720p-81f")
-    p.add_argument("--rope", choices=["fused", "pre"], default="pre")
+    p.add_argument("--rope", choices=["fused", "pre"], default="pre",
+                   help="pre: the RoPE pass rotates Q and K before the "
+                        "attention; fused: the attention kernel rotates in "
+                        "its tile stage (Q and K with --attn tiles; Q with "
+                        "--attn pair, K by the pass)")
+    p.add_argument("--attn", choices=["tiles", "pair"], default="tiles",
+                   help="self-attention kernel: two 128-row tiles per CTA, "
+                        "or CTA pairs (one MMA over two SMs)")
     p.add_argument("--impl", choices=["wan", "reference"], default="wan")
     p.add_argument("--parallel", choices=["replicas", "ulysses"],
                    default="replicas",
@@ -430,9 +437,11 @@ def causal_rooflines(dev, peak_tflops, reps=5):
 def attn_points(dev, pk, reps=6):
     """Self-attention launch alone at the two token counts of the metric:
     480p-81f (B 2 x 12 heads x 32,760 tokens) and 720p-81f (B 1 x 40 heads
-    x 75,600 tokens), each with Q / K rotated by the stand-alone RoPE pass
-    beforehand ("pre", the step's default) and with the rotation fused into
-    the attention kernel's tile stage ("fused").  CUDA events around `reps`
+    x 75,600 tokens).  Two-tile kernel with Q / K rotated beforehand ("pre")
+    and with the rotation of both fused into its tile stage ("fused"); the
+    CTA-pair kernel with Q / K rotated beforehand ("pair_pre") and with Q
+    rotated in its tile stage, K by the pass ("pair_fused_q"; the launch
+    timed here is the attention alone).  CUDA events around `reps`
     back-to-back launches on the launching stream after 2 warm-up launches;
     Q, K and V are each larger than L2 at 720p (774 MB) and together above
     it at 480p (3 x 201 MB).  FLOPs 4 * B * heads * L^2 * 128."""
@@ -459,15 +468,20 @@ def attn_points(dev, pk, reps=6):
         table = wan.rope3d_table(g)
         fl = 4.0 * B * H * L * L * 128
         point = {"tokens": L, "batch": B, "heads": H, "flops": fl}
-        for mode in ("pre", "fused"):
+        wan.rope3d_qk(None, k, g, table)  # k rotated once, for the pair
+        for mode in ("pre", "fused", "pair_pre", "pair_fused_q"):
             if mode == "pre":
-                wan.rope3d_qk(q, k, g, table)
-
                 def call():
                     wan.self_attn(q, k, v, o, g)
-            else:
+            elif mode == "fused":
                 def call():
                     wan.self_attn(q, k, v, o, g, table=table)
+            elif mode == "pair_pre":
+                def call():
+                    wan.self_attn_pair(q, k, v, o, g)
+            else:
+                def call():
+                    wan.self_attn_pair(q, k, v, o, g, table_q=table)
             for _ in range(2):
                 call()
             e0 = torch.cuda.Event(enable_timing=True)
@@ -555,18 +569,31 @@ def run_wan(args, w, rank, world, local_rank):
     ev_pairs = []
     ev_cross = []
 
+    def rope_pass(ds, strm=None):
+        # the stand-alone RoPE pass: Q and K (--rope pre), or K alone when
+        # the pair kernel rotates Q in its tile stage (--rope fused)
+        if args.rope == "pre":
+            wan.rope3d_qk(ds["q"], ds["k"], g, table, stream=strm)
+        elif args.attn == "pair":
+            wan.rope3d_qk(None, ds["k"], g, table, stream=strm)
+
+    def attention(ds, out, strm=None):
+        fused = table if args.rope == "fused" else None
+        if args.attn == "pair":
+            wan.self_attn_pair(ds["q"], ds["k"], ds["v"], out, g,
+                               table_q=fused, stream=strm)
+        else:
+            wan.self_attn(ds["q"], ds["k"], ds["v"], out, g, table=fused,
+                          stream=strm)
+
     def step(i, timed):
         s0, s1 = sigmas[i % w.steps], sigmas[i % w.steps + 1]
-        if args.rope == "pre":
-            wan.rope3d_qk(d["q"], d["k"], g, table)
+        rope_pass(d)
         if timed:
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-        if args.rope == "pre":
-            wan.self_attn(d["q"], d["k"], d["v"], o, g)
-        else:
-            wan.self_attn(d["q"], d["k"], d["v"], o, g, table=table)
+        attention(d, o)
         if timed:
             e1.record(stream)
             ev_pairs.append((e0, e1))
@@ -577,7 +604,8 @@ def run_wan(args, w, rank, world, local_rank):
             ev_cross.append((e1, e2))
         wan.fm_step(d["x"], d["v_cond"], d["v_uncond"], guide, s0, s1)
 
-    launches_per_step = 4 if args.rope == "pre" else 3
+    launches_per_step = 3 + (1 if args.rope == "pre" or args.attn == "pair"
+                             else 0)
 
     dist = None
     if world > 1:
@@ -659,13 +687,8 @@ def run_wan(args, w, rank, world, local_rank):
                 if read[bi] is not None:
                     comp.wait_event(read[bi])
                 s0, s1 = sigmas[i % w.steps], sigmas[i % w.steps + 1]
-                if args.rope == "pre":
-                    wan.rope3d_qk(ds["q"], ds["k"], g, table, stream=comp)
-                    wan.self_attn(ds["q"], ds["k"], ds["v"], os_[bi], g,
-                                  stream=comp)
-                else:
-                    wan.self_attn(ds["q"], ds["k"], ds["v"], os_[bi], g,
-                                  table=table, stream=comp)
+                rope_pass(ds, comp)
+                attention(ds, os_[bi], comp)
                 wan.cross_attn(os_[bi], ds["k_ctx"], ds["v_ctx"], ocs[bi],
                                lens, stream=comp)
                 wan.fm_step(ds["x"], ds["v_cond"], ds["v_uncond"], guide, s0,
@@ -721,6 +744,7 @@ def run_wan(args, w, rank, world, local_rank):
             "workload": w.name, "batch": B, "heads": H, "seq_len": L,
             "grid": [g.F, g.H, g.W], "text_tokens": w.text_tokens,
             "text_lens": lens, "latent": list(lat), "rope": args.rope,
+            "attn_kernel": args.attn,
             "parallelism": "replicas" if world > 1 else "single",
             "l2": "inputs larger than L2 (Q/K/V %.0f MB each)"
                   % (B * L * H * 256 / 1e6),
@@ -731,8 +755,10 @@ def run_wan(args, w, rank, world, local_rank):
             "measured_sustained": value / peak,
         },
         "roofline": {
-            "kernel": "attn_fwd_kernel self-attention" + (
-                "" if args.rope == "pre" else " with fused RoPE"),
+            "kernel": ("attn_pair_kernel (CTA pairs)" if args.attn == "pair"
+                       else "attn_fwd_kernel (two tiles per CTA)")
+            + " self-attention" + ("" if args.rope == "pre"
+                                   else " with fused RoPE"),
             "bound": "tensor", "achieved": achieved, "peak": peak,
             "unit": "TFLOP/s", "frac": achieved / peak,
             "traffic": ATTN_DRAM_PER_ALG_BYTE * 4 * B * L * H * 256,

@@ -115,16 +115,20 @@ int wan_self_attn(const void* q, const void* k, const void* v, void* o,
                   int B, wan_grid_t g, int heads, int head_dim,
                   const void* d_table, float softmax_scale, void* s);
 
-/* The same full self-attention (q and k already rotated) computed by pairs
- * of CTAs on two SMs: one tcgen05 MMA (cta_group::2) covers 256 query rows,
- * 128 in each SM's tensor memory, with each SM staging half of every K / V
- * block; three score slots per SM let the Q K^T of later blocks run while
- * the softmax of an earlier one is still going.  Same layouts, arguments,
- * errors and results as wan_self_attn with d_table == NULL.  Source: Wan2.2
- * source reading, ch. 4 "Full forward of one block" and ch. 8.            */
+/* The same full self-attention computed by pairs of CTAs on two SMs: one
+ * tcgen05 MMA (cta_group::2) covers 256 query rows, 128 in each SM's tensor
+ * memory, with each SM staging half of every K / V block; three score slots
+ * per SM let the Q K^T of later blocks run while the softmax of an earlier
+ * one is still going.  k must already be rotated (wan_rope3d_qk with a NULL
+ * q rotates k alone).  If d_table_q is NULL, q is used as given (already
+ * rotated); otherwise q is rotated by the 3D RoPE in shared memory, once per
+ * query tile, before the tensor cores read it (q in memory is untouched).
+ * Otherwise the same layouts, arguments, errors and results as
+ * wan_self_attn.  Source: Wan2.2 source reading, ch. 4 "Full forward of one
+ * block", "3D RoPE" and ch. 8.                                             */
 int wan_self_attn_pair(const void* q, const void* k, const void* v, void* o,
                        int B, wan_grid_t g, int heads, int head_dim,
-                       float softmax_scale, void* s);
+                       const void* d_table_q, float softmax_scale, void* s);
 
 /* ------------------------------------------------------ cross-attention --
  * Wan2.2 source reading, ch. 3 "Where did the prompt go" (each prompt is
@@ -168,6 +172,12 @@ int wan_block_causal_attn_pair(const void* q, const void* k, const void* v,
                                void* o, int B, int Lq, int Lk, int heads,
                                int head_dim, int chunk_tokens, int q_offset,
                                float softmax_scale, void* s);
+
+/* How many CTA pairs of the pair kernels can be resident at once on the
+ * current device (clusters of two CTAs must share a GPC, so an SM left over
+ * in a GPC with an odd number of SMs runs none).  A diagnostic; returns a
+ * negative wan_status on failure.                                          */
+int wan_attn_pair_resident_clusters(void);
 
 /* ---------------------------------------- block prologue and epilogue --
  * Wan2.2 source reading, ch. 4, section "Full forward of one block": the

@@ -83,6 +83,28 @@ def test_pair_7800_full_and_equals_reference_kernel_layout():
     assert_heads_close(map_threads(one, range(w.heads)), "pair 7800")
 
 
+@pytest.mark.parametrize("grid,B,H", [((3, 7, 13), 2, 3), ((5, 10, 20), 1, 2),
+                                      ((21, 6, 8), 1, 4)])
+def test_pair_rotates_q_in_kernel(grid, B, H):
+    # k rotated by the stand-alone pass (k alone), q in the kernel's tile
+    # stage; compared with the oracle's rotation of both
+    L = grid[0] * grid[1] * grid[2]
+    q, k, v = _qkv(B, L, H, 5100 + L)
+    g = wan.grid(*grid)
+    table = wan.rope3d_table(g)
+    qg, kg, vg = cuda(q), cuda(k), cuda(v)
+    wan.rope3d_qk(None, kg, g, table)
+    o, buf, guard = guarded_empty_like(qg)
+    wan.self_attn_pair(qg, kg, vg, o, g, table_q=table)
+    torch.cuda.synchronize()
+    assert wan.device_status() == 0
+    check_guards(buf, guard)
+    assert torch.equal(qg.cpu(), q)        # q in memory is untouched
+    want = oattn.attention(orope.rope3d(f64(q), grid),
+                           orope.rope3d(f64(k), grid), f64(v), scale_for())
+    assert_attn_close(f64(o), want, "pair rope-q L=%d" % L)
+
+
 def test_pair_deterministic():
     q, k, v = _qkv(1, 1000, 2, 77)
     a = _run(q, k, v, (5, 10, 20))

@@ -1356,7 +1356,7 @@ int wan_self_attn(const void* q, const void* k, const void* v, void* o,
 
 int wan_self_attn_pair(const void* q, const void* k, const void* v, void* o,
                        int B, wan_grid_t g, int heads, int head_dim,
-                       float softmax_scale, void* s) {
+                       const void* d_table_q, float softmax_scale, void* s) {
   using namespace wan;
   if (g.F < 1 || g.H < 1 || g.W < 1) return WAN_EINVAL;
   const int64_t L64 = static_cast<int64_t>(g.F) * g.H * g.W;
@@ -1364,6 +1364,10 @@ int wan_self_attn_pair(const void* q, const void* k, const void* v, void* o,
   const int L = static_cast<int>(L64);
   int st = check_common(q, k, v, o, B, L, L, heads, head_dim, softmax_scale);
   if (st != WAN_OK) return st;
+  if (d_table_q) {
+    if (wan_rope3d_table_bytes(g, head_dim) == 0) return WAN_EINVAL;
+    if (!aligned16(d_table_q)) return WAN_EALIGN;
+  }
   st = check_device(nullptr);
   if (st != WAN_OK) return st;
   CUtensorMap mq, mk, mv;
@@ -1372,7 +1376,7 @@ int wan_self_attn_pair(const void* q, const void* k, const void* v, void* o,
   if ((st = make_map_bf16(&mv, v, B, L, heads, 128)) != WAN_OK) return st;
   AttnArgs a;
   a.o = static_cast<__nv_bfloat16*>(o);
-  a.table = nullptr;
+  a.table = static_cast<const float4*>(d_table_q);
   a.Lq = L;
   a.Lk = L;
   a.heads = heads;
@@ -1383,7 +1387,34 @@ int wan_self_attn_pair(const void* q, const void* k, const void* v, void* o,
   a.cross = 0;
   a.chunk = 0;
   a.q_offset = 0;
-  return launch_pair<0>(mq, mk, mv, a, B, as_stream(s));
+  return d_table_q ? launch_pair<1>(mq, mk, mv, a, B, as_stream(s))
+                   : launch_pair<0>(mq, mk, mv, a, B, as_stream(s));
+}
+
+int wan_attn_pair_resident_clusters(void) {
+  using namespace wan;
+  int st = check_device(nullptr);
+  if (st != WAN_OK) return st;
+  if (cudaFuncSetAttribute(attn_pair_kernel<0>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           pair::SMEM) != cudaSuccess)
+    return WAN_ECUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2, 1, 1);
+  cfg.blockDim = dim3(pair::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = pair::SMEM;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeClusterDimension;
+  attr.val.clusterDim.x = 2;
+  attr.val.clusterDim.y = 1;
+  attr.val.clusterDim.z = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, attn_pair_kernel<0>, &cfg) !=
+      cudaSuccess)
+    return WAN_ECUDA;
+  return n;
 }
 
 int wan_block_causal_attn_pair(const void* q, const void* k, const void* v,

@@ -67,7 +67,7 @@ _SIGNATURES = {
     "wan_rope3d_qk": (_I, [_P, _P, _I, Grid, _I, _I, _P, _P]),
     "wan_self_attn": (_I, [_P, _P, _P, _P, _I, Grid, _I, _I, _P,
                            ctypes.c_float, _P]),
-    "wan_self_attn_pair": (_I, [_P, _P, _P, _P, _I, Grid, _I, _I,
+    "wan_self_attn_pair": (_I, [_P, _P, _P, _P, _I, Grid, _I, _I, _P,
                                 ctypes.c_float, _P]),
     "wan_cross_attn": (_I, [_P, _P, _P, _P, ctypes.POINTER(ctypes.c_int32),
                             _I, _I, _I, _I, _I, ctypes.c_float, _P]),
@@ -89,6 +89,7 @@ _SIGNATURES = {
                             ctypes.c_int64, _D, _I, _I, _P]),
     "wan_transpose_blocks": (_I, [_P, _P, ctypes.c_int64, ctypes.c_int64,
                                   ctypes.c_int64, _P]),
+    "wan_attn_pair_resident_clusters": (_I, []),
     "wan_wait_selftest": (_I, [_I, _P]),
     "wan_device_status": (_I, [_I]),
 }
@@ -276,9 +277,11 @@ def self_attn(q, k, v, o, g, table=None, softmax_scale=None, stream=None):
            "wan_self_attn")
 
 
-def self_attn_pair(q, k, v, o, g, softmax_scale=None, stream=None):
-    """o = softmax(q k^T * scale) v over the grid's tokens (q, k already
-    rotated), computed by the CTA-pair kernel (one MMA over two SMs)."""
+def self_attn_pair(q, k, v, o, g, table_q=None, softmax_scale=None,
+                   stream=None):
+    """o = softmax(rope(q) k^T * scale) v over the grid's tokens, computed by
+    the CTA-pair kernel (one MMA over two SMs).  k already rotated; q rotated
+    in the kernel if table_q is given, else used as given."""
     for name, t in (("q", q), ("k", k), ("v", v), ("o", o)):
         _bf16_bl(t, name)
         _shape_is(t, q.shape, name)
@@ -286,12 +289,13 @@ def self_attn_pair(q, k, v, o, g, softmax_scale=None, stream=None):
     if L != _grid_tokens(g):
         raise ValueError("q holds %d tokens, grid %r has %d"
                          % (L, g, _grid_tokens(g)))
-    _on_cuda(("q", q), ("k", k), ("v", v), ("o", o))
+    _check_table(table_q, g, D, "table_q")
+    _on_cuda(("q", q), ("k", k), ("v", v), ("o", o), ("table_q", table_q))
     if softmax_scale is None:
         softmax_scale = 1.0 / math.sqrt(D)
     _check(lib().wan_self_attn_pair(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, g,
-                                    H, D, softmax_scale, _stream(stream)),
-           "wan_self_attn_pair")
+                                    H, D, _ptr(table_q), softmax_scale,
+                                    _stream(stream)), "wan_self_attn_pair")
 
 
 def cross_attn(q, k_ctx, v_ctx, o, ctx_lens, softmax_scale=None,
@@ -468,6 +472,14 @@ def transpose_blocks(inp, out, a, b, row_bytes, stream=None):
     _check(lib().wan_transpose_blocks(_ptr(inp), _ptr(out), int(a), int(b),
                                       int(row_bytes), _stream(stream)),
            "wan_transpose_blocks")
+
+
+def attn_pair_resident_clusters():
+    """CTA pairs of the pair kernels resident at once on this device."""
+    n = lib().wan_attn_pair_resident_clusters()
+    if n < 0:
+        _check(n, "wan_attn_pair_resident_clusters")
+    return n
 
 
 def wait_selftest(arrive, stream=None):
