@@ -39,11 +39,14 @@ def parse():
     p.add_argument("--steps", type=int, default=10)
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--workload", default="720p-81f")
-    p.add_argument("--rope", choices=["fused", "pre"], default="pre",
+    p.add_argument("--rope", choices=["fused", "fused-q", "pre"],
+                   default="pre",
                    help="pre: the RoPE pass rotates Q and K before the "
-                        "attention; fused: the attention kernel rotates in "
-                        "its tile stage (Q and K with --attn tiles; Q with "
-                        "--attn pair, K by the pass)")
+                        "attention; fused: the attention kernel rotates Q "
+                        "and K in its tile stage (--attn tiles); fused-q: "
+                        "the pass rotates K alone and the kernel rotates Q "
+                        "in its tile stage (with --attn pair, fused means "
+                        "fused-q)")
     p.add_argument("--attn", choices=["tiles", "pair"], default="tiles",
                    help="self-attention kernel: two 128-row tiles per CTA, "
                         "or CTA pairs (one MMA over two SMs)")
@@ -437,9 +440,11 @@ def causal_rooflines(dev, peak_tflops, reps=5):
 def attn_points(dev, pk, reps=6):
     """Self-attention launch alone at the two token counts of the metric:
     480p-81f (B 2 x 12 heads x 32,760 tokens) and 720p-81f (B 1 x 40 heads
-    x 75,600 tokens).  Two-tile kernel with Q / K rotated beforehand ("pre")
-    and with the rotation of both fused into its tile stage ("fused"); the
-    CTA-pair kernel with Q / K rotated beforehand ("pair_pre") and with Q
+    x 75,600 tokens).  Two-tile kernel with Q / K rotated beforehand ("pre"),
+    with the rotation of both fused into its tile stage ("fused"), and with
+    Q rotated in its tile stage, K by the pass ("fused_q"; the launch timed
+    is the attention alone, the K pass moves half the bytes of the full
+    pass); the CTA-pair kernel with Q / K rotated beforehand ("pair_pre") and with Q
     rotated in its tile stage, K by the pass ("pair_fused_q"; the launch
     timed here is the attention alone).  CUDA events around `reps`
     back-to-back launches on the launching stream after 2 warm-up launches;
@@ -469,13 +474,16 @@ def attn_points(dev, pk, reps=6):
         fl = 4.0 * B * H * L * L * 128
         point = {"tokens": L, "batch": B, "heads": H, "flops": fl}
         wan.rope3d_qk(None, k, g, table)  # k rotated once, for the pair
-        for mode in ("pre", "fused", "pair_pre", "pair_fused_q"):
+        for mode in ("pre", "fused", "fused_q", "pair_pre", "pair_fused_q"):
             if mode == "pre":
                 def call():
                     wan.self_attn(q, k, v, o, g)
             elif mode == "fused":
                 def call():
                     wan.self_attn(q, k, v, o, g, table=table)
+            elif mode == "fused_q":
+                def call():
+                    wan.self_attn_rope_q(q, k, v, o, g, table)
             elif mode == "pair_pre":
                 def call():
                     wan.self_attn_pair(q, k, v, o, g)
@@ -569,21 +577,28 @@ def run_wan(args, w, rank, world, local_rank):
     ev_pairs = []
     ev_cross = []
 
+    rope_q = args.rope == "fused-q" or (args.rope == "fused"
+                                         and args.attn == "pair")
+
     def rope_pass(ds, strm=None):
         # the stand-alone RoPE pass: Q and K (--rope pre), or K alone when
-        # the pair kernel rotates Q in its tile stage (--rope fused)
+        # the attention kernel rotates Q in its tile stage
         if args.rope == "pre":
             wan.rope3d_qk(ds["q"], ds["k"], g, table, stream=strm)
-        elif args.attn == "pair":
+        elif rope_q:
             wan.rope3d_qk(None, ds["k"], g, table, stream=strm)
 
     def attention(ds, out, strm=None):
-        fused = table if args.rope == "fused" else None
         if args.attn == "pair":
             wan.self_attn_pair(ds["q"], ds["k"], ds["v"], out, g,
-                               table_q=fused, stream=strm)
+                               table_q=table if rope_q else None,
+                               stream=strm)
+        elif rope_q:
+            wan.self_attn_rope_q(ds["q"], ds["k"], ds["v"], out, g, table,
+                                 stream=strm)
         else:
-            wan.self_attn(ds["q"], ds["k"], ds["v"], out, g, table=fused,
+            wan.self_attn(ds["q"], ds["k"], ds["v"], out, g,
+                          table=table if args.rope == "fused" else None,
                           stream=strm)
 
     def step(i, timed):
@@ -604,8 +619,7 @@ def run_wan(args, w, rank, world, local_rank):
             ev_cross.append((e1, e2))
         wan.fm_step(d["x"], d["v_cond"], d["v_uncond"], guide, s0, s1)
 
-    launches_per_step = 3 + (1 if args.rope == "pre" or args.attn == "pair"
-                             else 0)
+    launches_per_step = 3 + (1 if args.rope == "pre" or rope_q else 0)
 
     dist = None
     if world > 1:
@@ -757,8 +771,9 @@ def run_wan(args, w, rank, world, local_rank):
         "roofline": {
             "kernel": ("attn_pair_kernel (CTA pairs)" if args.attn == "pair"
                        else "attn_fwd_kernel (two tiles per CTA)")
-            + " self-attention" + ("" if args.rope == "pre"
-                                   else " with fused RoPE"),
+            + " self-attention" + {"pre": "", "fused": " with fused RoPE",
+                                   "fused-q": " with Q rotated in the tile "
+                                   "stage"}[args.rope],
             "bound": "tensor", "achieved": achieved, "peak": peak,
             "unit": "TFLOP/s", "frac": achieved / peak,
             "traffic": ATTN_DRAM_PER_ALG_BYTE * 4 * B * L * H * 256,

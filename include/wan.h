@@ -115,6 +115,19 @@ int wan_self_attn(const void* q, const void* k, const void* v, void* o,
                   int B, wan_grid_t g, int heads, int head_dim,
                   const void* d_table, float softmax_scale, void* s);
 
+/* Self-attention with q rotated by the 3D RoPE in the attention kernel's
+ * tile stage (once per 256-row query tile, in shared memory; q in memory is
+ * untouched) and k already rotated -- e.g. by wan_rope3d_qk with a NULL q,
+ * or by wan_qk_norm_rope, which writes the rotated k anyway.  Rotating k in
+ * the tile stage (wan_self_attn with a table) repeats the rotation of every
+ * key block in every query tile; this form rotates each key once.  d_table
+ * is required.  Otherwise the same layouts, arguments, errors and results
+ * as wan_self_attn.  Source: Wan2.2 source reading, ch. 4 "3D RoPE".       */
+int wan_self_attn_rope_q(const void* q, const void* k, const void* v,
+                         void* o, int B, wan_grid_t g, int heads,
+                         int head_dim, const void* d_table,
+                         float softmax_scale, void* s);
+
 /* The same full self-attention computed by pairs of CTAs on two SMs: one
  * tcgen05 MMA (cta_group::2) covers 256 query rows, 128 in each SM's tensor
  * memory, with each SM staging half of every K / V block; three score slots

@@ -30,7 +30,7 @@ def _qkv(B, L, H, seed, q_scale=1.0):
 
 def _run_self(q, k, v, grid, mode):
     """mode: 'fused' (table in the kernel), 'pre' (wan_rope3d_qk first),
-    'none' (no RoPE)."""
+    'rope_q' (k by the pass, q in the kernel), 'none' (no RoPE)."""
     g = wan.grid(*grid)
     qg, kg, vg = cuda(q), cuda(k), cuda(v)
     o, buf, guard = guarded_empty_like(qg)
@@ -38,6 +38,12 @@ def _run_self(q, k, v, grid, mode):
     if mode == "pre":
         wan.rope3d_qk(qg, kg, g, table)
         wan.self_attn(qg, kg, vg, o, g)
+    elif mode == "rope_q":
+        # k by the pass, q in the kernel's tile stage (q stays unrotated)
+        wan.rope3d_qk(None, kg, g, table)
+        wan.self_attn_rope_q(qg, kg, vg, o, g, table)
+        torch.cuda.synchronize()
+        assert torch.equal(qg.cpu(), q)
     else:
         wan.self_attn(qg, kg, vg, o, g, table=table if mode == "fused"
                       else None)
@@ -67,7 +73,7 @@ SELF_CASES = [
 
 
 @pytest.mark.parametrize("grid,B,H", SELF_CASES)
-@pytest.mark.parametrize("mode", ["fused", "pre", "none"])
+@pytest.mark.parametrize("mode", ["fused", "pre", "rope_q", "none"])
 def test_self_attn_small(grid, B, H, mode):
     L = grid[0] * grid[1] * grid[2]
     q, k, v = _qkv(B, L, H, 100 + L)
@@ -76,7 +82,7 @@ def test_self_attn_small(grid, B, H, mode):
     assert_attn_close(got, want, "self %s %s" % (grid, mode))
 
 
-@pytest.mark.parametrize("mode", ["fused", "pre"])
+@pytest.mark.parametrize("mode", ["fused", "pre", "rope_q"])
 def test_self_attn_480p_17f(mode):
     # 17 frames at 480p: 5 x 30 x 52 = 7,800 tokens, 12 heads (full compare)
     grid, B, H = (5, 30, 52), 1, 12

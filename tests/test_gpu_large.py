@@ -56,6 +56,9 @@ def _sampled_self_parity(widx, n_rows, mode):
     if mode == "pre":
         wan.rope3d_qk(qg, kg, g, table)
         wan.self_attn(qg, kg, vg, o, g)
+    elif mode == "rope_q":
+        wan.rope3d_qk(None, kg, g, table)
+        wan.self_attn_rope_q(qg, kg, vg, o, g, table)
     else:
         wan.self_attn(qg, kg, vg, o, g, table=table)
     torch.cuda.synchronize()
@@ -95,6 +98,10 @@ def test_self_attn_720p_81f_sampled():
 
 def test_self_attn_720p_81f_prerotated_sampled():
     _sampled_self_parity(3, _rows(), "pre")
+
+
+def test_self_attn_720p_81f_rope_q_sampled():
+    _sampled_self_parity(3, _rows(), "rope_q")
 
 
 def test_self_attn_480p_165f_sampled():

@@ -33,8 +33,9 @@
 //              work there, or FMA work on another sub-partition, does not
 //              slow it), so the 16 MMAs that follow each softmax sit on the
 //              tile's critical path.  A second issuer warp measured slower.
-//   warps 10-11  RoPE variant: rotate the Q tiles and every K tile in shared
-//              memory before the tensor cores read them.
+//   warps 10-11  RoPE variants: rotate the Q tiles (kRope 1 and 2) and every
+//              K tile (kRope 1) in shared memory before the tensor cores read
+//              them; with kRope 2, K comes in rotated by the RoPE pass.
 // Tensor memory (512 columns): S/P of tile 0 at 0, of tile 1 at 128, O of
 // tile 0 at 256, of tile 1 at 384.  Operand tiles are [128 rows][128 ch]
 // bf16 stored as two 64-channel halves of [128][128 B] with the 128-byte
@@ -77,6 +78,11 @@ constexpr int KPP = BN / 16 / NPART;         // P V K-steps per part
 static_assert(BN % (32 * NPART) == 0, "parts of whole 32-key chunks");
 // Pairs (2e, 2e+1) with (e & 7) < kEmuPer8 take the FMA-pipe exponential.
 constexpr int kEmuPer8 = 2;
+// The same for the CTA-pair kernel's softmax.
+#ifndef WAN_PAIR_EMU8
+#define WAN_PAIR_EMU8 2
+#endif
+constexpr int kPairEmu8 = WAN_PAIR_EMU8;
 
 constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, BN, 0);   // K-major B
 constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, HD, 1);  // MN-major B
@@ -296,7 +302,7 @@ __device__ __forceinline__ float rowmax(const float* s) {
 // `pcol` (64 columns), sum of p returned.  kEmu: use the FMA-pipe
 // exponential for part of the pairs (never for a masked block, whose -inf
 // entries must give exact zeros).
-template <bool kEmu>
+template <bool kEmu, int kEmu8 = kEmuPer8>
 __device__ __forceinline__ void exp_store_chunks(const float* s, float c2,
                                                  float m, uint32_t pcol,
                                                  float2 (&acc)[4], int c0,
@@ -315,7 +321,7 @@ __device__ __forceinline__ void exp_store_chunks(const float* s, float c2,
       const float2 x =
           ffma2(make_float2(s[2 * pair], s[2 * pair + 1]), c22, nm2);
       float2 p;
-      if (kEmu && (pair & 7) < kEmuPer8) {
+      if (kEmu && (pair & 7) < kEmu8) {
         p = exp2_fma2(x);
       } else {
         p.x = ex2(x.x);
@@ -560,7 +566,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = ready_v(g - 1, j - 1, c.kv_len) && pv(0, g - 1, j - 1, n);
             if (!ok) break;
           }
-          ok = wait_warp(&bar[(kRope ? B_KREADY : B_KFULL) + sk],
+          ok = wait_warp(&bar[(kRope == 1 ? B_KREADY : B_KFULL) + sk],
                          (g / NSK) & 1, abort_flag, status);
           if (!ok) break;
           tc_fence_after();
@@ -610,7 +616,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         fence_proxy_async_smem();
         mbar_arrive(&bar[B_QREADY]);
-        for (int j = 0; j < c.nblk && ok; ++j) {
+        // kRope == 2: K comes in already rotated; only Q is rotated here
+        for (int j = 0; j < (kRope == 1 ? c.nblk : 0) && ok; ++j) {
           const int g = g0 + j, sk = g % NSK;
           ok = wait_warp(&bar[B_KFULL + sk], (g / NSK) & 1, abort_flag,
                          status);
@@ -930,8 +937,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(
       if (j < nblk) {
         const int sk = j % KSTAGES;
         if (j >= KSTAGES)
-          ok = wait_warp_cl(&bar[KEMPTY + sk], ((j / KSTAGES) - 1) & 1,
-                            abort_flag, status);
+          ok = wait_warp(&bar[KEMPTY + sk], ((j / KSTAGES) - 1) & 1,
+                         abort_flag, status);
         if (!ok) break;
         if (el) {
           const int key0 = j * BN + static_cast<int>(rank) * 64;
@@ -948,8 +955,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(
       if (jv >= 0) {
         const int sv = jv % VSTAGES;
         if (jv >= VSTAGES)
-          ok = wait_warp_cl(&bar[VEMPTY + sv], ((jv / VSTAGES) - 1) & 1,
-                            abort_flag, status);
+          ok = wait_warp(&bar[VEMPTY + sv], ((jv / VSTAGES) - 1) & 1,
+                         abort_flag, status);
         if (!ok) break;
         if (el) {
           mbar_expect_tx(&bar[VFULL + sv], VTILE);
@@ -971,8 +978,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(
   } else if (warp == 9 && !lead) {
     // ----------------------------------- CTA 1: forward load completions --
     auto fwd = [&](int full, int peer, uint32_t parity) -> bool {
-      if (!wait_warp_cl(&bar[full], parity, abort_flag, status)) return false;
-      if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&bar[peer]), 0));
+      if (!wait_warp(&bar[full], parity, abort_flag, status)) return false;
+      if (lane == 0)
+        mbar_arrive_remote_relaxed(mapa_shared(smem_u32(&bar[peer]), 0));
       __syncwarp();
       return true;
     };
@@ -985,7 +993,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(
         ok = fwd(VFULL + jv % VSTAGES, VPEER + jv % VSTAGES, (jv / VSTAGES) & 1);
     }
     // every MMA of the pair is done before this CTA's memory is released
-    wait_warp_cl_drain(&bar[DRAIN], 0, status);
+    wait_warp_drain(&bar[DRAIN], 0, status);
   } else if (warp == 9) {
     // ---------------------------------------------- CTA 0: MMA issuer --
     const uint64_t dq = sdesc_sw128(smem_u32(sQ), 16, 1024);
@@ -994,13 +1002,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(
     const uint64_t dv = sdesc_sw128(smem_u32(sV), 16, 1024);
     const bool el = elect_one();
     bool ok =
-        wait_warp_cl(&bar[kRopeQ ? QREADY : QFULL], 0, abort_flag, status) &&
+        wait_warp(&bar[kRopeQ ? QREADY : QFULL], 0, abort_flag, status) &&
         wait_warp_cl(&bar[QPEER], 0, abort_flag, status);
     // S(j) = Q K(j)^T into slot j % NSLOT of both CTAs.
     auto issue_s = [&](int j) -> bool {
       const int sk = j % KSTAGES;
       const uint32_t ph = (j / KSTAGES) & 1;
-      if (!wait_warp_cl(&bar[KFULL + sk], ph, abort_flag, status) ||
+      if (!wait_warp(&bar[KFULL + sk], ph, abort_flag, status) ||
           !wait_warp_cl(&bar[KPEER + sk], ph, abort_flag, status))
         return false;
       tc_fence_after();
@@ -1025,7 +1033,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(
       const uint32_t pv = (j / VSTAGES) & 1;
       ok = wait_warp_cl(&bar[PREADY + sl], (j / NSLOT) & 1, abort_flag,
                         status) &&
-           wait_warp_cl(&bar[VFULL + sv], pv, abort_flag, status) &&
+           wait_warp(&bar[VFULL + sv], pv, abort_flag, status) &&
            wait_warp_cl(&bar[VPEER + sv], pv, abort_flag, status);
       if (!ok) break;
       tc_fence_after();
@@ -1049,11 +1057,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(
     if (ok && el) umma_commit_pair(&bar[OFINAL], BOTH);
     if (el) umma_commit_pair(&bar[DRAIN], BOTH);
     __syncwarp();
-    wait_warp_cl_drain(&bar[DRAIN], 0, status);
+    wait_warp_drain(&bar[DRAIN], 0, status);
   } else if (kRopeQ && warp >= 10) {
     // ------------------------------------------------ Q rotation (RoPE) --
     const int tr = threadIdx.x - 320;  // 0..63
-    if (wait_warp_cl(&bar[QFULL], 0, abort_flag, status)) {
+    if (wait_warp(&bar[QFULL], 0, abort_flag, status)) {
       for (int rr = tr; rr < RM; rr += 64)
         if (q0 + rr < args.Lq) rope_row(sQ, rr, q0 + rr, args);
       fence_proxy_async_smem();
@@ -1078,8 +1086,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(
     bool ok = true;
     for (int j = 0; j < nblk && ok; ++j) {
       const int sl = j % NSLOT;
-      ok = wait_warp_cl(&bar[SFULL + sl], (j / NSLOT) & 1, abort_flag,
-                        status);
+      ok = wait_warp(&bar[SFULL + sl], (j / NSLOT) & 1, abort_flag, status);
       if (!ok) break;
       tc_fence_after();
       const uint32_t s_col = lane_base + TM_SLOT0 + sl * 128 + 64 * h;
@@ -1112,8 +1119,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(
         if (__any_sync(0xffffffffu, need)) {
           const float m_new = need ? mx : m_run;
           const float alpha = ex2(m_run - m_new);
-          ok = wait_warp_cl(&bar[PVDONE + (j - 1) % NSLOT],
-                            ((j - 1) / NSLOT) & 1, abort_flag, status);
+          ok = wait_warp(&bar[PVDONE + (j - 1) % NSLOT],
+                         ((j - 1) / NSLOT) & 1, abort_flag, status);
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
@@ -1140,16 +1147,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(
       if (masked)
         exp_store_chunks<false>(s, c2, m_run, s_col, acc, 0, 2);
       else
-        exp_store_chunks<true>(s, c2, m_run, s_col, acc, 0, 2);
+        exp_store_chunks<true, kPairEmu8>(s, c2, m_run, s_col, acc, 0, 2);
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0)
-        mbar_arrive_cluster(mapa_shared(smem_u32(&bar[PREADY + sl]), 0));
+      if (lane == 0) {
+        if (lead)
+          mbar_arrive(&bar[PREADY + sl]);
+        else
+          mbar_arrive_remote_relaxed(
+              mapa_shared(smem_u32(&bar[PREADY + sl]), 0));
+      }
       const float2 tsum = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
       l_run += tsum.x + tsum.y;
     }
-    if (ok) ok = wait_warp_cl(&bar[OFINAL], 0, abort_flag, status);
+    if (ok) ok = wait_warp(&bar[OFINAL], 0, abort_flag, status);
     if (ok) {
       // row sum over both key halves
       s_xch[nblk & 1][h][r] = l_run;
@@ -1352,6 +1364,42 @@ int wan_self_attn(const void* q, const void* k, const void* v, void* o,
   a.q_offset = 0;
   return d_table ? launch<1, 0>(mq, mk, mv, a, B, as_stream(s))
                  : launch<0, 0>(mq, mk, mv, a, B, as_stream(s));
+}
+
+int wan_self_attn_rope_q(const void* q, const void* k, const void* v,
+                         void* o, int B, wan_grid_t g, int heads,
+                         int head_dim, const void* d_table,
+                         float softmax_scale, void* s) {
+  using namespace wan;
+  if (!d_table) return WAN_EINVAL;
+  if (g.F < 1 || g.H < 1 || g.W < 1) return WAN_EINVAL;
+  const int64_t L64 = static_cast<int64_t>(g.F) * g.H * g.W;
+  if (L64 > (1 << 26)) return WAN_EINVAL;
+  const int L = static_cast<int>(L64);
+  int st = check_common(q, k, v, o, B, L, L, heads, head_dim, softmax_scale);
+  if (st != WAN_OK) return st;
+  if (wan_rope3d_table_bytes(g, head_dim) == 0) return WAN_EINVAL;
+  if (!aligned16(d_table)) return WAN_EALIGN;
+  st = check_device(nullptr);
+  if (st != WAN_OK) return st;
+  CUtensorMap mq, mk, mv;
+  if ((st = make_map_bf16(&mq, q, B, L, heads, BM)) != WAN_OK) return st;
+  if ((st = make_map_bf16(&mk, k, B, L, heads, BM)) != WAN_OK) return st;
+  if ((st = make_map_bf16(&mv, v, B, L, heads, BM)) != WAN_OK) return st;
+  AttnArgs a;
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.table = static_cast<const float4*>(d_table);
+  a.Lq = L;
+  a.Lk = L;
+  a.heads = heads;
+  a.F = g.F;
+  a.H = g.H;
+  a.W = g.W;
+  a.scale_log2 = softmax_scale * 1.4426950408889634f;
+  a.cross = 0;
+  a.chunk = 0;
+  a.q_offset = 0;
+  return launch<2, 0>(mq, mk, mv, a, B, as_stream(s));
 }
 
 int wan_self_attn_pair(const void* q, const void* k, const void* v, void* o,

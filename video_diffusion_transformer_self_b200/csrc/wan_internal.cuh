@@ -469,6 +469,19 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
       : "memory");
 }
 
+// Relaxed arrive on a peer CTA's mbarrier (no release fence: a release at
+// cluster scope stalls the arriving warp for about 1,600 cycles).  Used
+// only where what the arrival announces is already complete before it is
+// issued: tensor-memory stores after tcgen05.wait::st, or a TMA load whose
+// local barrier phase has been observed.
+__device__ __forceinline__ void mbar_arrive_remote_relaxed(
+    uint32_t cluster_addr) {
+  asm volatile(
+      "mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(
+          cluster_addr)
+      : "memory");
+}
+
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar,
                                                       uint32_t parity) {
   uint32_t ok;

@@ -67,6 +67,8 @@ _SIGNATURES = {
     "wan_rope3d_qk": (_I, [_P, _P, _I, Grid, _I, _I, _P, _P]),
     "wan_self_attn": (_I, [_P, _P, _P, _P, _I, Grid, _I, _I, _P,
                            ctypes.c_float, _P]),
+    "wan_self_attn_rope_q": (_I, [_P, _P, _P, _P, _I, Grid, _I, _I, _P,
+                                  ctypes.c_float, _P]),
     "wan_self_attn_pair": (_I, [_P, _P, _P, _P, _I, Grid, _I, _I, _P,
                                 ctypes.c_float, _P]),
     "wan_cross_attn": (_I, [_P, _P, _P, _P, ctypes.POINTER(ctypes.c_int32),
@@ -275,6 +277,29 @@ def self_attn(q, k, v, o, g, table=None, softmax_scale=None, stream=None):
     _check(lib().wan_self_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, g, H, D,
                                _ptr(table), softmax_scale, _stream(stream)),
            "wan_self_attn")
+
+
+def self_attn_rope_q(q, k, v, o, g, table, softmax_scale=None,
+                     stream=None):
+    """o = softmax(rope(q) k^T * scale) v: q rotated in the attention
+    kernel's tile stage, k already rotated (e.g. rope3d_qk(None, k, ...))."""
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o)):
+        _bf16_bl(t, name)
+        _shape_is(t, q.shape, name)
+    B, L, H, D = q.shape
+    if L != _grid_tokens(g):
+        raise ValueError("q holds %d tokens, grid %r has %d"
+                         % (L, g, _grid_tokens(g)))
+    if table is None:
+        raise ValueError("self_attn_rope_q needs a table")
+    _check_table(table, g, D)
+    _on_cuda(("q", q), ("k", k), ("v", v), ("o", o), ("table", table))
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(D)
+    _check(lib().wan_self_attn_rope_q(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B,
+                                      g, H, D, _ptr(table), softmax_scale,
+                                      _stream(stream)),
+           "wan_self_attn_rope_q")
 
 
 def self_attn_pair(q, k, v, o, g, table_q=None, softmax_scale=None,
