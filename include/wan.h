@@ -177,6 +177,43 @@ int wan_block_causal_attn(const void* q, const void* k, const void* v,
                           int head_dim, int chunk_tokens, int q_offset,
                           float softmax_scale, void* s);
 
+/* The same block-causal attention with each (256-row tile, head, batch row)
+ * work item's key blocks cut into n_split consecutive ranges run as separate
+ * CTAs, followed by a combining pass.  When every query of the call sees the
+ * same keys (a KV-cache step over the whole cache) the items are equal, and
+ * their count can leave the last wave of CTAs mostly idle (760 items on 148
+ * SMs is 5.1 waves); n_split ranges make n_split times as many shorter
+ * items.  Each range writes its rows' unnormalised fp32 O and (row max, row
+ * sum) into `workspace`; the combining pass rescales and sums them, the
+ * online-softmax step of the kernel applied across ranges, and writes bf16
+ * o.  The result equals wan_block_causal_attn's up to fp32 summation order.
+ * n_split in [1, 8] and at most the key-block count of the lightest item
+ * (WAN_EINVAL otherwise); n_split == 1 is wan_block_causal_attn.
+ * workspace: caller-owned device memory of at least
+ * wan_block_causal_attn_workspace_bytes(B, Lq, heads, n_split) bytes,
+ * 16-byte aligned (NULL allowed when that is 0); its contents on entry do
+ * not matter and on return are unspecified.  Calls that share a workspace
+ * must not overlap on the device.                                         */
+int wan_block_causal_attn_split(const void* q, const void* k, const void* v,
+                                void* o, int B, int Lq, int Lk, int heads,
+                                int head_dim, int chunk_tokens, int q_offset,
+                                float softmax_scale, int n_split,
+                                void* workspace, size_t workspace_bytes,
+                                void* s);
+
+/* Workspace bytes of wan_block_causal_attn_split: n_split * B * Lq * heads
+ * * (128 * 4 + 8) for n_split > 1, 0 for n_split == 1 or bad arguments.    */
+size_t wan_block_causal_attn_workspace_bytes(int B, int Lq, int heads,
+                                             int n_split);
+
+/* Host: the key-range count wan_block_causal_attn_split is fastest with on
+ * the current device: 1 unless every item sees the same keys; otherwise the
+ * smallest count (up to 4, at least 8 key blocks per range) whose waves of
+ * CTAs are at least 95 % full, else the fullest.  Negative wan_status on
+ * bad arguments.                                                           */
+int wan_block_causal_attn_splits(int B, int Lq, int Lk, int heads,
+                                 int chunk_tokens, int q_offset);
+
 /* The same block-causal attention computed by pairs of CTAs on two SMs (the
  * kernel of wan_self_attn_pair, with the per-row key limit above; the
  * 256-row tiles of each head run heaviest first).  Same arguments, layouts,

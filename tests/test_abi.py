@@ -171,3 +171,43 @@ def test_argument_checks_without_device(lib):
     assert L.wan_transpose_blocks(None, None, 0, 3, 16, None) == wan.WAN_OK
     assert L.wan_transpose_blocks(None, big_o, 2, 3, 16, None) \
         == wan.WAN_EINVAL
+
+
+def test_split_block_causal_host_checks(lib):
+    # workspace size: n_split * rows * (512 + 8) bytes, 0 without a split
+    assert lib.wan_block_causal_attn_workspace_bytes(1, 4680, 40, 1) == 0
+    assert lib.wan_block_causal_attn_workspace_bytes(1, 4680, 40, 3) == \
+        3 * 4680 * 40 * 520
+    assert lib.wan_block_causal_attn_workspace_bytes(2, 10, 3, 2) == \
+        2 * 2 * 10 * 3 * 520
+    assert lib.wan_block_causal_attn_workspace_bytes(1, 10, 2, 9) == 0
+    assert lib.wan_block_causal_attn_workspace_bytes(0, 10, 2, 2) == 0
+    p = ctypes.c_void_p(4096)
+    o = ctypes.c_void_p(8192)
+    ws = ctypes.c_void_p(1 << 24)
+    need = lib.wan_block_causal_attn_workspace_bytes(1, 600, 2, 2)
+    L = lib
+    # n_split out of range
+    assert L.wan_block_causal_attn_split(p, p, p, o, 1, 600, 600, 2, 128,
+                                         120, 0, 0.1, 0, ws, need, None) \
+        == wan.WAN_EINVAL
+    assert L.wan_block_causal_attn_split(p, p, p, o, 1, 600, 600, 2, 128,
+                                         120, 0, 0.1, 9, ws, need, None) \
+        == wan.WAN_EINVAL
+    # the lightest item (the first 256 queries, keys < 256) has 2 key
+    # blocks: 3 ranges would leave one empty
+    assert L.wan_block_causal_attn_split(p, p, p, o, 1, 600, 600, 2, 128,
+                                         128, 0, 0.1, 3, ws, 1 << 20, None) \
+        == wan.WAN_EINVAL
+    # workspace missing, too small, misaligned
+    assert L.wan_block_causal_attn_split(p, p, p, o, 1, 600, 600, 2, 128,
+                                         120, 0, 0.1, 2, None, need, None) \
+        == wan.WAN_EINVAL
+    assert L.wan_block_causal_attn_split(p, p, p, o, 1, 600, 600, 2, 128,
+                                         120, 0, 0.1, 2, ws, need - 1, None) \
+        == wan.WAN_EINVAL
+    assert L.wan_block_causal_attn_split(p, p, p, o, 1, 600, 600, 2, 128,
+                                         120, 0, 0.1, 2,
+                                         ctypes.c_void_p((1 << 24) + 8),
+                                         need, None) == wan.WAN_EALIGN
+    assert L.wan_block_causal_attn_splits(1, 10, 5, 2, 4, 0) == wan.WAN_EINVAL

@@ -67,6 +67,35 @@ def test_kv_cache_chunk_step(chunk, n_chunks, pair):
     assert_attn_close(got, want, "kv-cache chunk %d" % chunk)
 
 
+@pytest.mark.parametrize("L,chunk,q_offset,Lq,n_split", [
+    (600, 120, 480, 120, 2),     # KV-cache step, equal items
+    (600, 120, 480, 120, 3),
+    (1000, 100, 700, 300, 4),    # KV-cache step over 3 chunks, 2 tiles
+    (700, 128, 0, 700, 2),       # full sequence: early rows see no key of
+                                 # the second range (row max stays -inf)
+    (520, 200, 0, 520, 2),       # chunk boundaries mid-block
+])
+def test_split_key_ranges(L, chunk, q_offset, Lq, n_split):
+    q, k, v = _qkv(2, L, L, 2, 1300 + L + n_split)
+    ql = q[:, q_offset:q_offset + Lq].contiguous()
+    qg, kg, vg = cuda(ql), cuda(k), cuda(v)
+    o, buf, guard = guarded_empty_like(qg)
+    ws = torch.full((wan.block_causal_workspace_bytes(2, Lq, 2, n_split),),
+                    255, dtype=torch.uint8, device="cuda")  # NaN-patterned
+    wan.block_causal_attn(qg, kg, vg, o, chunk, q_offset, split=n_split,
+                          workspace=ws)
+    torch.cuda.synchronize()
+    assert wan.device_status() == 0
+    check_guards(buf, guard)
+    want = oattn.block_causal_attention(f64(ql), f64(k), f64(v), scale_for(),
+                                        chunk, q_offset)
+    got = f64(o)
+    assert_attn_close(got, want, "split %d L=%d" % (n_split, L))
+    # the same as one key range, up to fp32 summation order
+    one = _run(ql, k, v, chunk, q_offset)
+    assert np.max(np.abs(got - one)) <= 1e-2
+
+
 @pytest.mark.parametrize("pair", [False, True], ids=["tiles", "pair"])
 def test_first_chunk_ignores_later_keys(pair):
     chunk, L = 96, 400
@@ -137,5 +166,23 @@ def test_kv_cache_last_chunk_480p_165f_sampled(pair):
     q0 = FULL_L - FULL_CHUNK
     ql = q[:, q0:].contiguous()
     got = _run(ql, k, v, FULL_CHUNK, q0, pair=pair)
+    rows = _rows(FULL_CHUNK, 92, [1, FULL_CHUNK - 2])
+    _per_head(got, ql, k, v, rows, q0, "480p-165f KV step")
+
+
+def test_kv_cache_last_chunk_480p_165f_split_sampled():
+    # the launch bench.py times: key ranges chosen for this device (3 on
+    # 148 SMs: 760 equal items would fill 5.1 waves), combining pass after
+    q, k, v = _full_qkv()
+    q0 = FULL_L - FULL_CHUNK
+    ql = q[:, q0:].contiguous()
+    n = wan.block_causal_splits(1, FULL_CHUNK, FULL_L, FULL_H, FULL_CHUNK, q0)
+    assert n > 1
+    qg, kg, vg = cuda(ql), cuda(k), cuda(v)
+    o = torch.empty_like(qg)
+    wan.block_causal_attn(qg, kg, vg, o, FULL_CHUNK, q0, split="auto")
+    torch.cuda.synchronize()
+    assert wan.device_status() == 0
+    got = f64(o)
     rows = _rows(FULL_CHUNK, 92, [1, FULL_CHUNK - 2])
     _per_head(got, ql, k, v, rows, q0, "480p-165f KV step")

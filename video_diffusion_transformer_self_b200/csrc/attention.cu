@@ -97,20 +97,28 @@ struct AttnArgs {
   int chunk;            // > 0: block-causal, chunk length in tokens
   int q_offset;         // block-causal: absolute position of query row 0
   int n_tiles_x;        // 256-row query tile pairs per (head, batch row)
-  int items;            // n_tiles_x * heads * B work items
+  int items;            // n_tiles_x * heads * B * n_split work items
+  int n_split = 1;             // key ranges per (tile pair, head, batch)
+  float* part_o = nullptr;     // n_split > 1: unnormalised O per key range,
+  float2* part_ml = nullptr;   //   fp32 [split][B][Lq][heads][128], and
+  int64_t split_rows = 0;      //   (row max, row sum); B * Lq * heads rows
   int lens[MAX_CROSS_BATCH];
 };
 
-// One work item: a pair of 128-row query tiles of one (head, batch row).
-// Items are numbered tile-fastest, then head, then batch row, the order a
-// (tiles, heads, B) grid launches in; block-causal items run heaviest first
-// within a head.
+// One work item: a pair of 128-row query tiles of one (head, batch row),
+// and with n_split > 1 one of n_split consecutive ranges of its key blocks.
+// Items are numbered key range fastest, then tile, then head, then batch
+// row; block-causal items run heaviest first within a head.
 struct Item {
   int q0, head, b, kv_len, nblk;
+  int kb0;    // first key block of the item's range
+  int split;  // index of the key range
 };
 
 __device__ __forceinline__ Item item_of(const AttnArgs& a, int it) {
   Item c;
+  c.split = it % a.n_split;
+  it /= a.n_split;
   const int tx = it % a.n_tiles_x;
   const int rest = it / a.n_tiles_x;
   c.head = rest % a.heads;
@@ -124,7 +132,9 @@ __device__ __forceinline__ Item item_of(const AttnArgs& a, int it) {
     kv = min(a.Lk, (last / a.chunk + 1) * a.chunk);
   }
   c.kv_len = kv;
-  c.nblk = (kv + BN - 1) / BN;
+  const int nb = (kv + BN - 1) / BN;
+  c.kb0 = c.split * nb / a.n_split;
+  c.nblk = (c.split + 1) * nb / a.n_split - c.kb0;
   return c;
 }
 
@@ -434,9 +444,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (leader) {
             mbar_expect_tx(&bar[B_KFULL + sk], TILE);
             tma_load_4d(sK + sk * TILE, &tm_k, &bar[B_KFULL + sk], 0, c.head,
-                        j * BN, c.b);
+                        (c.kb0 + j) * BN, c.b);
             tma_load_4d(sK + sk * TILE + HALF, &tm_k, &bar[B_KFULL + sk], 64,
-                        c.head, j * BN, c.b);
+                        c.head, (c.kb0 + j) * BN, c.b);
           }
           ++nk;
           const int sv = g % NSV, uv = g / NSV;
@@ -447,9 +457,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (leader) {
             mbar_expect_tx(&bar[B_VFULL + sv], TILE);
             tma_load_4d(sV + sv * TILE, &tm_v, &bar[B_VFULL + sv], 0, c.head,
-                        j * BN, c.b);
+                        (c.kb0 + j) * BN, c.b);
             tma_load_4d(sV + sv * TILE + HALF, &tm_v, &bar[B_VFULL + sv], 64,
-                        c.head, j * BN, c.b);
+                        c.head, (c.kb0 + j) * BN, c.b);
           }
           ++nv;
           __syncwarp();
@@ -663,7 +673,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         static_assert(BN == 128, "one 128-column TMEM load per score row");
         tmem_ld128(s_col, s);
         tmem_ld_wait128(s);
-        const int lim = row_lim - j * BN;  // valid keys of this row here
+        const int lim = row_lim - (cur.kb0 + j) * BN;  // valid keys here
         // warp-uniform: any masked row sends the warp down the exact path
         const bool masked = __any_sync(0xffffffffu, lim < BN);
         if (masked) {
@@ -717,9 +727,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr int CPP = BN / 32 / NPART;  // 32-key chunks per part
 #pragma unroll
         for (int part = 0; part < NPART; ++part) {
+          // A row with no visible key yet (possible in a later key range
+          // of a block-causal item) keeps m = -inf: its scores are all -inf
+          // and exponentiate against 0 to exact zeros.
           if (masked)
-            exp_store_chunks<false>(s, c2, m_run, s_col, acc, part * CPP,
-                                    (part + 1) * CPP);
+            exp_store_chunks<false>(s, c2, m_run == -INFINITY ? 0.f : m_run,
+                                    s_col, acc, part * CPP, (part + 1) * CPP);
           else
             exp_store_chunks<true>(s, c2, m_run, s_col, acc, part * CPP,
                                    (part + 1) * CPP);
@@ -739,11 +752,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Item ce = item_of(args, it_e);
         const float inv = 1.0f / l_run;
         const int row = ce.q0 + t * BM + r;
-        __nv_bfloat16* orow =
-            args.o + ((static_cast<int64_t>(ce.b) * args.Lq + row) *
-                          args.heads + ce.head) * HD;
+        const int64_t orow_i =
+            (static_cast<int64_t>(ce.b) * args.Lq + row) * args.heads + ce.head;
+        __nv_bfloat16* orow = args.o + orow_i * HD;
+        if (args.n_split > 1) {
+          // one key range of the row: unnormalised O and (row max, row sum)
+          // for the combining pass
+          const int64_t prow = ce.split * args.split_rows + orow_i;
+          float4* dst = reinterpret_cast<float4*>(args.part_o + prow * HD);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+          for (int c = 0; c < 4; ++c) {
+            float o[32];
+            tmem_ld32(o_col + c * 32, o);
+            tmem_ld_wait32(o);
+            if (row < args.Lq) {
+#pragma unroll
+              for (int e = 0; e < 8; ++e)
+                dst[c * 8 + e] = make_float4(o[4 * e], o[4 * e + 1],
+                                             o[4 * e + 2], o[4 * e + 3]);
+            }
+          }
+          if (row < args.Lq) args.part_ml[prow] = make_float2(m_run, l_run);
+        }
+#pragma unroll
+        for (int c = 0; c < (args.n_split > 1 ? 0 : 4); ++c) {
           float o[32];
           tmem_ld32(o_col + c * 32, o);
           tmem_ld_wait32(o);
@@ -1207,6 +1239,44 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(
   }
 }
 
+// Combining pass of a split key range: for each output row (b, token,
+// head), the n_split partial results (unnormalised O_s, row max m_s in log2
+// units, row sum l_s) give O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s,
+// M = max_s m_s -- the same online-softmax rescaling the kernel applies
+// between key blocks.  One warp per row, 4 channels per lane.
+__global__ void __launch_bounds__(256)
+    combine_splits_kernel(const float4* __restrict__ part_o,
+                          const float2* __restrict__ part_ml,
+                          __nv_bfloat16* __restrict__ o, int64_t rows,
+                          int n_split) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) +
+                     (threadIdx.x >> 5);
+       row < rows; row += warps) {
+    float mmax = -INFINITY;
+    for (int sp = 0; sp < n_split; ++sp)
+      mmax = fmaxf(mmax, part_ml[sp * rows + row].x);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float l = 0.f;
+    for (int sp = 0; sp < n_split; ++sp) {
+      const float2 ml = part_ml[sp * rows + row];
+      const float w = ml.x == -INFINITY ? 0.f : ex2(ml.x - mmax);
+      const float4 v = part_o[(sp * rows + row) * (HD / 4) + lane];
+      acc.x = fmaf(w, v.x, acc.x);
+      acc.y = fmaf(w, v.y, acc.y);
+      acc.z = fmaf(w, v.z, acc.z);
+      acc.w = fmaf(w, v.w, acc.w);
+      l = fmaf(w, ml.y, l);
+    }
+    const float inv = 1.0f / l;
+    uint2 out;
+    out.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+    out.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+    reinterpret_cast<uint2*>(o + row * HD)[lane] = out;
+  }
+}
+
 // One warp waits, with the same bounded wait the attention kernel uses, on
 // an mbarrier that needs one arrival and receives `arrive` (0 or 1).  With
 // none the wait runs out after kWaitLimitNs, records WAN_ETIMEOUT in the
@@ -1262,7 +1332,8 @@ int launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
     if (state[dev] != 1) return WAN_EUNSUPPORTED;
   }
   a.n_tiles_x = (a.Lq + QT * BM - 1) / (QT * BM);
-  const int64_t items = static_cast<int64_t>(a.n_tiles_x) * a.heads * B;
+  const int64_t items =
+      static_cast<int64_t>(a.n_tiles_x) * a.heads * B * a.n_split;
   if (items > INT32_MAX) return WAN_EINVAL;
   a.items = static_cast<int>(items);
   // One CTA per item, except cross-attention: its items are short (a few
@@ -1321,6 +1392,25 @@ int check_common(const void* q, const void* k, const void* v, void* o, int B,
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
     return WAN_EALIGN;
   if (o == q || o == k || o == v) return WAN_EINVAL;
+  return WAN_OK;
+}
+
+
+// Key limit of the last query row of two-tile item `tile` (block-causal).
+int causal_item_kv(int tile, int Lq, int Lk, int chunk, int q_offset) {
+  const int last = min((tile + 1) * QT * BM, Lq) - 1 + q_offset;
+  return min(Lk, (last / chunk + 1) * chunk);
+}
+
+int causal_check(const void* q, const void* k, const void* v, void* o, int B,
+                 int Lq, int Lk, int heads, int head_dim, int chunk_tokens,
+                 int q_offset, float softmax_scale) {
+  int st = check_common(q, k, v, o, B, Lq, Lk, heads, head_dim,
+                        softmax_scale);
+  if (st != WAN_OK) return st;
+  if (chunk_tokens < 1 || q_offset < 0 ||
+      static_cast<int64_t>(q_offset) + Lq > Lk)
+    return WAN_EINVAL;
   return WAN_OK;
 }
 
@@ -1437,6 +1527,108 @@ int wan_self_attn_pair(const void* q, const void* k, const void* v, void* o,
   a.q_offset = 0;
   return d_table_q ? launch_pair<1>(mq, mk, mv, a, B, as_stream(s))
                    : launch_pair<0>(mq, mk, mv, a, B, as_stream(s));
+}
+
+
+size_t wan_block_causal_attn_workspace_bytes(int B, int Lq, int heads,
+                                             int n_split) {
+  if (B < 1 || Lq < 1 || heads < 1 || n_split < 1 || n_split > 8) return 0;
+  if (n_split == 1) return 0;
+  return static_cast<size_t>(n_split) * B * Lq * heads *
+         (wan::HD * sizeof(float) + 2 * sizeof(float));
+}
+
+int wan_block_causal_attn_splits(int B, int Lq, int Lk, int heads,
+                                 int chunk_tokens, int q_offset) {
+  using namespace wan;
+  if (B < 1 || Lq < 1 || Lk < 1 || heads < 1 || chunk_tokens < 1 ||
+      q_offset < 0 || static_cast<int64_t>(q_offset) + Lq > Lk)
+    return WAN_EINVAL;
+  int dev = 0;
+  int st = check_device(&dev);
+  if (st != WAN_OK) return st;
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+      cudaSuccess)
+    return WAN_ECUDA;
+  const int tiles = (Lq + QT * BM - 1) / (QT * BM);
+  const int kv_first = causal_item_kv(0, Lq, Lk, chunk_tokens, q_offset);
+  const int kv_last =
+      causal_item_kv(tiles - 1, Lq, Lk, chunk_tokens, q_offset);
+  // Unequal items already run heaviest first; equal ones (a KV-cache step,
+  // where every query sees the whole cache) are split when their count
+  // leaves the last wave of CTAs partly empty.
+  if (kv_first != kv_last) return 1;
+  const int nblk = (kv_first + BN - 1) / BN;
+  const double items = static_cast<double>(tiles) * heads * B;
+  int best = 1;
+  double best_eff = 0.0;
+  for (int sp = 1; sp <= 4; ++sp) {
+    if (sp > 1 && nblk < 8 * sp) break;  // at least 8 key blocks per range
+    const double waves = items * sp / sms;
+    const double eff = waves / ceil(waves);
+    if (eff > best_eff + 0.01) {
+      best = sp;
+      best_eff = eff;
+    }
+    if (eff >= 0.95) break;
+  }
+  return best;
+}
+
+int wan_block_causal_attn_split(const void* q, const void* k, const void* v,
+                                void* o, int B, int Lq, int Lk, int heads,
+                                int head_dim, int chunk_tokens, int q_offset,
+                                float softmax_scale, int n_split,
+                                void* workspace, size_t workspace_bytes,
+                                void* s) {
+  using namespace wan;
+  int st = causal_check(q, k, v, o, B, Lq, Lk, heads, head_dim, chunk_tokens,
+                        q_offset, softmax_scale);
+  if (st != WAN_OK) return st;
+  if (n_split < 1 || n_split > 8) return WAN_EINVAL;
+  if (n_split > 1) {
+    // every key range of every item holds at least one key block
+    const int kv0 = causal_item_kv(0, Lq, Lk, chunk_tokens, q_offset);
+    if ((kv0 + BN - 1) / BN < n_split) return WAN_EINVAL;
+    const size_t need =
+        wan_block_causal_attn_workspace_bytes(B, Lq, heads, n_split);
+    if (!workspace || workspace_bytes < need) return WAN_EINVAL;
+    if (!aligned16(workspace)) return WAN_EALIGN;
+  }
+  st = check_device(nullptr);
+  if (st != WAN_OK) return st;
+  CUtensorMap mq, mk, mv;
+  if ((st = make_map_bf16(&mq, q, B, Lq, heads, BM)) != WAN_OK) return st;
+  if ((st = make_map_bf16(&mk, k, B, Lk, heads, BM)) != WAN_OK) return st;
+  if ((st = make_map_bf16(&mv, v, B, Lk, heads, BM)) != WAN_OK) return st;
+  AttnArgs a;
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.table = nullptr;
+  a.Lq = Lq;
+  a.Lk = Lk;
+  a.heads = heads;
+  a.F = a.H = a.W = 1;
+  a.scale_log2 = softmax_scale * 1.4426950408889634f;
+  a.cross = 0;
+  a.chunk = chunk_tokens;
+  a.q_offset = q_offset;
+  a.n_split = n_split;
+  const int64_t rows = static_cast<int64_t>(B) * Lq * heads;
+  if (n_split > 1) {
+    a.part_o = static_cast<float*>(workspace);
+    a.part_ml = reinterpret_cast<float2*>(a.part_o + n_split * rows * HD);
+    a.split_rows = rows;
+  }
+  cudaStream_t cs = as_stream(s);
+  st = launch<0, 0>(mq, mk, mv, a, B, cs);
+  if (st != WAN_OK || n_split == 1) return st;
+  const int64_t blocks64 = (rows + 7) / 8;
+  const int blocks = static_cast<int>(blocks64 < 148 * 16 ? blocks64 : 148 * 16);
+  combine_splits_kernel<<<blocks, 256, 0, cs>>>(
+      reinterpret_cast<const float4*>(a.part_o), a.part_ml, a.o, rows,
+      n_split);
+  return cudaGetLastError() == cudaSuccess ? WAN_OK : WAN_ECUDA;
 }
 
 int wan_attn_pair_resident_clusters(void) {

@@ -77,6 +77,12 @@ _SIGNATURES = {
                                    _I, ctypes.c_float, _P]),
     "wan_block_causal_attn_pair": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I,
                                         _I, _I, ctypes.c_float, _P]),
+    "wan_block_causal_attn_split": (_I, [_P, _P, _P, _P, _I, _I, _I, _I,
+                                         _I, _I, _I, ctypes.c_float, _I, _P,
+                                         ctypes.c_size_t, _P]),
+    "wan_block_causal_attn_workspace_bytes": (ctypes.c_size_t,
+                                              [_I, _I, _I, _I]),
+    "wan_block_causal_attn_splits": (_I, [_I, _I, _I, _I, _I, _I]),
     "wan_adaln_modulate": (_I, [_P, _P, _P, _P, _I, _I, _I, ctypes.c_float,
                                 _P]),
     "wan_qk_norm_rope": (_I, [_P, _P, _P, _P, _I, Grid, _I, _I, _P,
@@ -346,10 +352,15 @@ def cross_attn(q, k_ctx, v_ctx, o, ctx_lens, softmax_scale=None,
 
 
 def block_causal_attn(q, k, v, o, chunk_tokens, q_offset=0,
-                      softmax_scale=None, stream=None, pair=False):
+                      softmax_scale=None, stream=None, pair=False,
+                      split=None, workspace=None):
     """Chunk-wise causal attention: query a = q_offset + i sees keys
     j < (a // chunk_tokens + 1) * chunk_tokens (and j < Lk).  pair=True runs
-    the CTA-pair kernel (wan_block_causal_attn_pair)."""
+    the CTA-pair kernel (wan_block_causal_attn_pair).  split: None (one key
+    range per item), "auto" (wan_block_causal_attn_splits) or a count; with
+    more than one range the call needs a workspace (a CUDA tensor of at
+    least block_causal_workspace_bytes(...) bytes), allocated here with
+    torch if not given."""
     for name, t in (("q", q), ("k", k), ("v", v), ("o", o)):
         _bf16_bl(t, name)
     B, Lq, H, D = q.shape
@@ -360,11 +371,48 @@ def block_causal_attn(q, k, v, o, chunk_tokens, q_offset=0,
     _on_cuda(("q", q), ("k", k), ("v", v), ("o", o))
     if softmax_scale is None:
         softmax_scale = 1.0 / math.sqrt(D)
+    n_split = 1
+    if split == "auto":
+        n_split = block_causal_splits(B, Lq, Lk, H, chunk_tokens, q_offset)
+    elif split is not None:
+        n_split = int(split)
+    if n_split > 1:
+        if pair:
+            raise ValueError("key ranges run on the two-tile kernel only")
+        need = block_causal_workspace_bytes(B, Lq, H, n_split)
+        if workspace is None:
+            import torch
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        if not workspace.is_contiguous() or \
+                workspace.numel() * workspace.element_size() < need:
+            raise ValueError("workspace must be a contiguous tensor of at "
+                             "least %d bytes" % need)
+        _on_cuda(("q", q), ("workspace", workspace))
+        _check(lib().wan_block_causal_attn_split(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(o), B, Lq, Lk, H, D,
+            int(chunk_tokens), int(q_offset), softmax_scale, n_split,
+            _ptr(workspace), workspace.numel() * workspace.element_size(),
+            _stream(stream)), "wan_block_causal_attn_split")
+        return
     fn = lib().wan_block_causal_attn_pair if pair else \
         lib().wan_block_causal_attn
     _check(fn(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, Lq, Lk, H, D,
               int(chunk_tokens), int(q_offset), softmax_scale,
               _stream(stream)), "wan_block_causal_attn")
+
+
+def block_causal_workspace_bytes(B, Lq, heads, n_split):
+    """Workspace bytes of the split block-causal call."""
+    return lib().wan_block_causal_attn_workspace_bytes(B, Lq, heads, n_split)
+
+
+def block_causal_splits(B, Lq, Lk, heads, chunk_tokens, q_offset=0):
+    """Key-range count the split block-causal call is fastest with."""
+    n = lib().wan_block_causal_attn_splits(B, Lq, Lk, heads,
+                                           int(chunk_tokens), int(q_offset))
+    if n < 1:
+        _check(n, "wan_block_causal_attn_splits")
+    return n
 
 
 def _f32(t, name):
