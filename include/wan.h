@@ -52,7 +52,9 @@ enum wan_status {
   WAN_EALIGN = -2,        /* pointer not 16-byte aligned                   */
   WAN_EUNSUPPORTED = -3,  /* current device is not sm_100 (B200 class)     */
   WAN_ECUDA = -4,         /* a CUDA runtime call or launch failed          */
-  WAN_ETIMEOUT = -5       /* a bounded in-kernel wait ran out              */
+  WAN_ETIMEOUT = -5,      /* a bounded in-kernel wait ran out              */
+  WAN_ENOSPACE = -6       /* needs more scratch than the library's fixed
+                             array holds (the no-allocation call)          */
 };
 
 /* Static text of a status code (never NULL). */
@@ -213,6 +215,35 @@ size_t wan_block_causal_attn_workspace_bytes(int B, int Lq, int heads,
  * bad arguments.                                                           */
 int wan_block_causal_attn_splits(int B, int Lq, int Lk, int heads,
                                  int chunk_tokens, int q_offset);
+
+/* wan_block_causal_attn_split for callers that cannot allocate device
+ * memory: the pages have no counterpart of this call.  Some callers must
+ * not allocate once they run -- a serving loop whose memory is fixed at
+ * start-up (an allocation can synchronise the device and stall the other
+ * streams), or code embedded in a host application that owns all device
+ * memory and offers no allocator -- and so cannot provide the workspace.
+ * This call takes its scratch from a fixed array in device memory instead:
+ * 64 MiB (wan_block_causal_attn_noalloc_max_bytes()), created on each GPU
+ * that loads the library and held until the process exits.  Calls whose
+ * wan_block_causal_attn_workspace_bytes(B, Lq, heads, n_split) exceeds it
+ * return WAN_ENOSPACE without touching the device.  The first call on a
+ * device looks up the array's device address (with that device current)
+ * and keeps it; make that first call before any stream capture.  Every
+ * call on a device shares the one array, and it keeps the last call's
+ * contents; nothing in it needs to start at zero (each call writes every
+ * value it reads).  Calls that overlap on the GPU -- on different streams,
+ * or from different host threads -- race on the array and give wrong
+ * results; serialise them.  Arguments, results and other errors as
+ * wan_block_causal_attn_split, without the workspace arguments.           */
+int wan_block_causal_attn_split_noalloc(const void* q, const void* k,
+                                        const void* v, void* o, int B, int Lq,
+                                        int Lk, int heads, int head_dim,
+                                        int chunk_tokens, int q_offset,
+                                        float softmax_scale, int n_split,
+                                        void* s);
+
+/* Bytes of the fixed scratch array of wan_block_causal_attn_split_noalloc. */
+size_t wan_block_causal_attn_noalloc_max_bytes(void);
 
 /* The same block-causal attention computed by pairs of CTAs on two SMs (the
  * kernel of wan_self_attn_pair, with the per-row key limit above; the

@@ -1631,6 +1631,56 @@ int wan_block_causal_attn_split(const void* q, const void* k, const void* v,
   return cudaGetLastError() == cudaSuccess ? WAN_OK : WAN_ECUDA;
 }
 
+// ------------------------------------------------- without allocation --
+// Scratch of wan_block_causal_attn_split_noalloc: a fixed array in device
+// memory, created when the library is loaded on a device and held until the
+// process exits, so that the call needs no allocation.  Shared by every
+// call on that device.
+constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;  // 64 MiB
+static __device__ __align__(256) unsigned char
+    g_noalloc_scratch[kNoAllocScratchBytes];
+
+int wan_block_causal_attn_split_noalloc(const void* q, const void* k,
+                                        const void* v, void* o, int B, int Lq,
+                                        int Lk, int heads, int head_dim,
+                                        int chunk_tokens, int q_offset,
+                                        float softmax_scale, int n_split,
+                                        void* s) {
+  const size_t need =
+      wan_block_causal_attn_workspace_bytes(B, Lq, heads, n_split);
+  if (n_split > 1 && need == 0) return WAN_EINVAL;
+  if (need > kNoAllocScratchBytes) return WAN_ENOSPACE;
+  int dev = 0;
+  int st = wan::check_device(&dev);
+  if (st != WAN_OK) return st;
+  // Device address of the scratch array on this device: looked up once per
+  // device, with that device current (in host code the array's name is
+  // only a stand-in for it).
+  static std::mutex mu;
+  static void* addr[64];
+  void* ws = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+      void* ptr = nullptr;
+      if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess ||
+          !ptr)
+        return WAN_ECUDA;
+      addr[dev] = ptr;
+    }
+    ws = addr[dev];
+  }
+  return wan_block_causal_attn_split(q, k, v, o, B, Lq, Lk, heads, head_dim,
+                                     chunk_tokens, q_offset, softmax_scale,
+                                     n_split, n_split > 1 ? ws : nullptr,
+                                     n_split > 1 ? kNoAllocScratchBytes : 0,
+                                     s);
+}
+
+size_t wan_block_causal_attn_noalloc_max_bytes(void) {
+  return kNoAllocScratchBytes;
+}
+
 int wan_attn_pair_resident_clusters(void) {
   using namespace wan;
   int st = check_device(nullptr);

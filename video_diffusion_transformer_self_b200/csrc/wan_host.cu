@@ -95,6 +95,8 @@ const char* wan_status_string(int status) {
       return "CUDA runtime error";
     case WAN_ETIMEOUT:
       return "bounded in-kernel wait timed out";
+    case WAN_ENOSPACE:
+      return "needs more scratch than the library's fixed array holds";
     default:
       return "unknown status";
   }

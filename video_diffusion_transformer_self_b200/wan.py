@@ -21,6 +21,7 @@ WAN_EALIGN = -2
 WAN_EUNSUPPORTED = -3
 WAN_ECUDA = -4
 WAN_ETIMEOUT = -5
+WAN_ENOSPACE = -6
 
 
 class WanError(RuntimeError):
@@ -83,6 +84,10 @@ _SIGNATURES = {
     "wan_block_causal_attn_workspace_bytes": (ctypes.c_size_t,
                                               [_I, _I, _I, _I]),
     "wan_block_causal_attn_splits": (_I, [_I, _I, _I, _I, _I, _I]),
+    "wan_block_causal_attn_split_noalloc": (_I, [_P, _P, _P, _P, _I, _I, _I,
+                                                 _I, _I, _I, _I,
+                                                 ctypes.c_float, _I, _P]),
+    "wan_block_causal_attn_noalloc_max_bytes": (ctypes.c_size_t, []),
     "wan_adaln_modulate": (_I, [_P, _P, _P, _P, _I, _I, _I, ctypes.c_float,
                                 _P]),
     "wan_qk_norm_rope": (_I, [_P, _P, _P, _P, _I, Grid, _I, _I, _P,
