@@ -172,6 +172,8 @@ def _oracle_cross(q, kc, vc, lens):
     (3, 300, 512, 2, [1, 512, 129]),   # single key, full length, ragged
     (2, 129, 200, 1, [128, 200]),      # exactly one block; ragged 2nd block
     (1, 7, 5, 3, [5]),
+    (3, 19993, 512, 4, [37, 512, 300]),  # 948 items: each persistent CTA
+                                         # reuses its output staging buffer
 ])
 def test_cross_attn_small(B, Lq, Lk, H, lens):
     q, kc, vc = _cross_inputs(B, Lq, Lk, H, 300 + Lq, lens)

@@ -153,7 +153,9 @@ enum : int {
   B_OFREE = B_OFINAL + QT,   // per tile: O of the item read out (4 warps)
   B_QEMPTY = B_OFREE + QT,   // an item's S MMAs done: Q buffer reusable
   B_DRAIN = B_QEMPTY + 1,
-  NBAR = B_DRAIN + 1
+  B_OSTAGE = B_DRAIN + 1,    // per tile: output staging buffer free
+  B_OWRITTEN = B_OSTAGE + QT,  // per tile: staging written (4 warps)
+  NBAR = B_OWRITTEN + QT
 };
 
 // ------------------------------------------------------- small helpers --
@@ -352,7 +354,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v,
+                    const __grid_constant__ CUtensorMap tm_o,
                     const __grid_constant__ AttnArgs args) {
+  // Ring depths: cross-attention (kPersist) gives one K stage to a staging
+  // buffer for the output tile, which it writes with TMA stores.
+  constexpr int nsk = kPersist ? NSK - 1 : NSK;
+  constexpr int nsv = NSV;
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t bar[NBAR];
   __shared__ uint32_t s_tmem;
@@ -369,19 +376,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* sm = smem_raw + (((raw + 1023u) & ~1023u) - raw);
   uint8_t* sQ = sm;                   // QT tiles
-  uint8_t* sK = sm + QT * TILE;       // NSK tiles
-  uint8_t* sV = sK + NSK * TILE;      // NSV tiles
+  uint8_t* sK = sm + QT * TILE;       // nsk tiles
+  uint8_t* sV = sK + nsk * TILE;      // nsv tiles
+  uint8_t* sO = sV + nsv * TILE;      // kPersist: one [128][64] half per tile
 
   if (threadIdx.x == 0) {
     s_abort = 0;
     mbar_init(&bar[B_QFULL], 1);
     mbar_init(&bar[B_QREADY], kRopeThreads);
-    for (int i = 0; i < NSK; ++i) {
+    for (int i = 0; i < nsk; ++i) {
       mbar_init(&bar[B_KFULL + i], 1);
       mbar_init(&bar[B_KREADY + i], kRopeThreads);
       mbar_init(&bar[B_KEMPTY + i], 1);
     }
-    for (int i = 0; i < NSV; ++i) {
+    for (int i = 0; i < nsv; ++i) {
       mbar_init(&bar[B_VFULL + i], 1);
       mbar_init(&bar[B_VEMPTY + i], 1);
     }
@@ -391,6 +399,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&bar[B_PPART + t * NPART + q], 4);
       mbar_init(&bar[B_OFINAL + t], 1);
       mbar_init(&bar[B_OFREE + t], 4);
+      mbar_init(&bar[B_OSTAGE + t], 1);
+      mbar_init(&bar[B_OWRITTEN + t], 4);
     }
     mbar_init(&bar[B_QEMPTY], 1);
     mbar_init(&bar[B_DRAIN], 1);
@@ -436,7 +446,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++nq;
         for (int j = 0; j < c.nblk && ok; ++j) {
           const int g = nk;  // key blocks issued so far == this block's g
-          const int sk = g % NSK, uk = g / NSK;
+          const int sk = g % nsk, uk = g / nsk;
           if (uk > 0)
             ok = wait_warp(&bar[B_KEMPTY + sk], (uk - 1) & 1, abort_flag,
                            status);
@@ -449,7 +459,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         c.head, (c.kb0 + j) * BN, c.b);
           }
           ++nk;
-          const int sv = g % NSV, uv = g / NSV;
+          const int sv = g % nsv, uv = g / nsv;
           if (uv > 0)
             ok = wait_warp(&bar[B_VEMPTY + sv], (uv - 1) & 1, abort_flag,
                            status);
@@ -468,10 +478,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (*abort_flag) {
         // Let copies already issued land before the CTA leaves.
         if (nq > 0) wait_warp_drain(&bar[B_QFULL], (nq - 1) & 1, status);
-        for (int g = (nk > NSK ? nk - NSK : 0); g < nk; ++g)
-          wait_warp_drain(&bar[B_KFULL + g % NSK], (g / NSK) & 1, status);
-        for (int g = (nv > NSV ? nv - NSV : 0); g < nv; ++g)
-          wait_warp_drain(&bar[B_VFULL + g % NSV], (g / NSV) & 1, status);
+        for (int g = (nk > nsk ? nk - nsk : 0); g < nk; ++g)
+          wait_warp_drain(&bar[B_KFULL + g % nsk], (g / nsk) & 1, status);
+        for (int g = (nv > nsv ? nv - nsv : 0); g < nv; ++g)
+          wait_warp_drain(&bar[B_VFULL + g % nsv], (g / nsv) & 1, status);
       }
     } else if (warp == 9) {
       // -------------------------------------------------------- MMA issuer --
@@ -487,7 +497,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // arithmetic runs in all lanes (warp-uniform); one lane issues.
       auto issue_s = [&](int t, int g) {
         const uint64_t a0 = dq + ((t * TILE) >> 4);
-        const uint64_t b0 = dk + (((g % NSK) * TILE) >> 4);
+        const uint64_t b0 = dk + (((g % nsk) * TILE) >> 4);
         const uint32_t d = tmem + t * 128;
         if (leader) {
 #pragma unroll
@@ -504,7 +514,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // O_t += P_t V over the keys of P part `part`; g is the block's global
       // count (ring stage), jl its index within the item (accumulate flag).
       auto issue_pv_part = [&](int t, int g, int jl, int part) {
-        const uint64_t b0 = dv + (((g % NSV) * TILE) >> 4);
+        const uint64_t b0 = dv + (((g % nsv) * TILE) >> 4);
         const uint32_t d = tmem + TM_O + t * 128;
         const uint32_t a = tmem + t * 128;
         if (leader) {
@@ -527,12 +537,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       // Waits for V of block g and clears its text-padding rows: they may
       // hold anything (NaN included), and P is 0 there but 0 * NaN is not.
       auto ready_v = [&](int g, int jl, int kv_len) -> bool {
-        if (!wait_warp(&bar[B_VFULL + g % NSV], (g / NSV) & 1, abort_flag,
+        if (!wait_warp(&bar[B_VFULL + g % nsv], (g / nsv) & 1, abort_flag,
                        status))
           return false;
         if (args.cross && kv_len < (jl + 1) * BN) {
           const int first = kv_len - jl * BN;
-          uint8_t* vt = sV + (g % NSV) * TILE;
+          uint8_t* vt = sV + (g % nsv) * TILE;
           for (int idx = lane; idx < (BN - first) * 16; idx += 32) {
             const int r = first + (idx >> 4);
             const int c = idx & 15;
@@ -571,20 +581,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                        status);
         for (int j = 0; j < c.nblk && ok; ++j) {
           const int g = g0 + j;
-          const int sk = g % NSK;
+          const int sk = g % nsk;
           if (j > 0) {
             ok = ready_v(g - 1, j - 1, c.kv_len) && pv(0, g - 1, j - 1, n);
             if (!ok) break;
           }
           ok = wait_warp(&bar[(kRope == 1 ? B_KREADY : B_KFULL) + sk],
-                         (g / NSK) & 1, abort_flag, status);
+                         (g / nsk) & 1, abort_flag, status);
           if (!ok) break;
           tc_fence_after();
           issue_s(0, g);
           if (j > 0) {
             ok = pv(1, g - 1, j - 1, n);
             if (!ok) break;
-            commit(&bar[B_VEMPTY + (g - 1) % NSV]);
+            commit(&bar[B_VEMPTY + (g - 1) % nsv]);
           }
           issue_s(1, g);
           // the item's last S: the Q buffer is free once these are done
@@ -600,7 +610,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (ok) {
             commit(&bar[B_OFINAL + 1]);
-            commit(&bar[B_VEMPTY + g % NSV]);
+            commit(&bar[B_VEMPTY + g % nsv]);
           }
         }
         g0 += c.nblk;
@@ -628,8 +638,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(&bar[B_QREADY]);
         // kRope == 2: K comes in already rotated; only Q is rotated here
         for (int j = 0; j < (kRope == 1 ? c.nblk : 0) && ok; ++j) {
-          const int g = g0 + j, sk = g % NSK;
-          ok = wait_warp(&bar[B_KFULL + sk], (g / NSK) & 1, abort_flag,
+          const int g = g0 + j, sk = g % nsk;
+          ok = wait_warp(&bar[B_KFULL + sk], (g / nsk) & 1, abort_flag,
                          status);
           if (!ok) break;
           for (int rr = tr; rr < BN; rr += kRopeThreads)
@@ -755,7 +765,65 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int64_t orow_i =
             (static_cast<int64_t>(ce.b) * args.Lq + row) * args.heads + ce.head;
         __nv_bfloat16* orow = args.o + orow_i * HD;
-        if (args.n_split > 1) {
+        if (kPersist) {
+          // Output tile through shared memory and TMA stores, one 64-channel
+          // half at a time: each thread writes its row's 128 B into the
+          // tile's staging half (128-byte swizzle, the layout the tensor map
+          // stores from), and warp 4t's lane 0 issues the store.  A row per
+          // thread stored straight to global memory scatters every store
+          // instruction over 32 rows 10 KB apart and stalls the warps on
+          // the store queue; the next item's softmax then starts late.
+          uint8_t* stg = sO + t * HALF;
+          const bool issuer_warp = (warp & 3) == 0;
+#pragma unroll 1
+          for (int hc = 0; hc < 2; ++hc) {
+            const int use = 2 * n + hc;
+            if (issuer_warp) {
+              // the previous store from this buffer has read it
+              if (lane == 0) {
+                if (use > 0) bulk_wait_group_read0();
+                mbar_arrive(&bar[B_OSTAGE + t]);
+              }
+              __syncwarp();
+            }
+            const bool free_ok =
+                wait_warp(&bar[B_OSTAGE + t], use & 1, abort_flag, status);
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              float o[32];
+              tmem_ld32(o_col + hc * 64 + c * 32, o);
+              tmem_ld_wait32(o);
+              uint32_t pk[16];
+#pragma unroll
+              for (int e = 0; e < 16; ++e)
+                pk[e] = pack_bf16x2(o[2 * e] * inv, o[2 * e + 1] * inv);
+              if (free_ok) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const int cc = c * 4 + e;  // 16-byte chunk of the row
+                  *reinterpret_cast<uint4*>(stg + r * 128 +
+                                            ((cc ^ (r & 7)) << 4)) =
+                      make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2],
+                                 pk[4 * e + 3]);
+                }
+              }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar[B_OWRITTEN + t]);
+            if (issuer_warp) {
+              const bool written =
+                  wait_warp(&bar[B_OWRITTEN + t], use & 1, abort_flag, status);
+              if (written && lane == 0) {
+                tma_store_4d(&tm_o, stg, hc * 64, ce.head, ce.q0 + t * BM,
+                             ce.b);
+                bulk_commit_group();
+              }
+              __syncwarp();
+            }
+          }
+        }
+        if (!kPersist && args.n_split > 1) {
           // one key range of the row: unnormalised O and (row max, row sum)
           // for the combining pass
           const int64_t prow = ce.split * args.split_rows + orow_i;
@@ -775,7 +843,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (row < args.Lq) args.part_ml[prow] = make_float2(m_run, l_run);
         }
 #pragma unroll
-        for (int c = 0; c < (args.n_split > 1 ? 0 : 4); ++c) {
+        for (int c = 0; c < (kPersist || args.n_split > 1 ? 0 : 4); ++c) {
           float o[32];
           tmem_ld32(o_col + c * 32, o);
           tmem_ld_wait32(o);
@@ -799,6 +867,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
+  // the output stores of the staging buffers are complete before the CTA
+  // (and its shared memory) goes away
+  if (kPersist && warp < 8 && (warp & 3) == 0 && lane == 0) bulk_wait_group0();
   tc_fence_before();
   __syncthreads();
   if (warp == 9) {
@@ -1301,7 +1372,7 @@ __global__ void __launch_bounds__(32) wait_selftest_kernel(int arrive) {
 
 template <int kRope, int kPersist>
 int launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-           AttnArgs a, int B, cudaStream_t s) {
+           const CUtensorMap& mo, AttnArgs a, int B, cudaStream_t s) {
   static std::mutex mu;
   static int state[64];  // 0 unknown, 1 ready, 2 unusable
   int dev = 0;
@@ -1347,8 +1418,8 @@ int launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
       return WAN_ECUDA;
     grid = a.items < sms ? a.items : sms;
   }
-  attn_fwd_kernel<kRope, kPersist><<<grid, kThreads, SMEM_DYN, s>>>(mq, mk, mv,
-                                                                     a);
+  attn_fwd_kernel<kRope, kPersist><<<grid, kThreads, SMEM_DYN, s>>>(
+      mq, mk, mv, mo, a);
   return cudaGetLastError() == cudaSuccess ? WAN_OK : WAN_ECUDA;
 }
 
@@ -1452,8 +1523,8 @@ int wan_self_attn(const void* q, const void* k, const void* v, void* o,
   a.cross = 0;
   a.chunk = 0;
   a.q_offset = 0;
-  return d_table ? launch<1, 0>(mq, mk, mv, a, B, as_stream(s))
-                 : launch<0, 0>(mq, mk, mv, a, B, as_stream(s));
+  return d_table ? launch<1, 0>(mq, mk, mv, mq, a, B, as_stream(s))
+                 : launch<0, 0>(mq, mk, mv, mq, a, B, as_stream(s));
 }
 
 int wan_self_attn_rope_q(const void* q, const void* k, const void* v,
@@ -1489,7 +1560,7 @@ int wan_self_attn_rope_q(const void* q, const void* k, const void* v,
   a.cross = 0;
   a.chunk = 0;
   a.q_offset = 0;
-  return launch<2, 0>(mq, mk, mv, a, B, as_stream(s));
+  return launch<2, 0>(mq, mk, mv, mq, a, B, as_stream(s));
 }
 
 int wan_self_attn_pair(const void* q, const void* k, const void* v, void* o,
@@ -1621,7 +1692,7 @@ int wan_block_causal_attn_split(const void* q, const void* k, const void* v,
     a.split_rows = rows;
   }
   cudaStream_t cs = as_stream(s);
-  st = launch<0, 0>(mq, mk, mv, a, B, cs);
+  st = launch<0, 0>(mq, mk, mv, mq, a, B, cs);
   if (st != WAN_OK || n_split == 1) return st;
   const int64_t blocks64 = (rows + 7) / 8;
   const int blocks = static_cast<int>(blocks64 < 148 * 16 ? blocks64 : 148 * 16);
@@ -1766,7 +1837,7 @@ int wan_block_causal_attn(const void* q, const void* k, const void* v,
   a.cross = 0;
   a.chunk = chunk_tokens;
   a.q_offset = q_offset;
-  return launch<0, 0>(mq, mk, mv, a, B, as_stream(s));
+  return launch<0, 0>(mq, mk, mv, mq, a, B, as_stream(s));
 }
 
 int wan_cross_attn(const void* q, const void* k_ctx, const void* v_ctx,
@@ -1797,7 +1868,9 @@ int wan_cross_attn(const void* q, const void* k_ctx, const void* v_ctx,
   a.chunk = 0;
   a.q_offset = 0;
   for (int i = 0; i < B; ++i) a.lens[i] = ctx_lens[i];
-  return launch<0, 1>(mq, mk, mv, a, B, as_stream(s));
+  CUtensorMap mo;
+  if ((st = make_map_bf16(&mo, o, B, Lq, heads, BM)) != WAN_OK) return st;
+  return launch<0, 1>(mq, mk, mv, mo, a, B, as_stream(s));
 }
 
 int wan_wait_selftest(int arrive, void* s) {
