@@ -764,7 +764,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int row = ce.q0 + t * BM + r;
         const int64_t orow_i =
             (static_cast<int64_t>(ce.b) * args.Lq + row) * args.heads + ce.head;
-        __nv_bfloat16* orow = args.o + orow_i * HD;
         if (kPersist) {
           // Output tile through shared memory and TMA stores, one 64-channel
           // half at a time: each thread writes its row's 128 B into the
@@ -842,21 +841,43 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (row < args.Lq) args.part_ml[prow] = make_float2(m_run, l_run);
         }
+        if (!kPersist && args.n_split == 1) {
+          // One item per CTA: once the item's last P V is done (OFINAL_t),
+          // no MMA reads the K ring and no load fills it, so tile t's output
+          // is staged in K stage t (two 64-channel halves, 128-byte swizzle)
+          // and written by two TMA stores from warp 4t's lane 0.
+          uint8_t* stg = sK + t * TILE;
 #pragma unroll
-        for (int c = 0; c < (kPersist || args.n_split > 1 ? 0 : 4); ++c) {
-          float o[32];
-          tmem_ld32(o_col + c * 32, o);
-          tmem_ld_wait32(o);
-          uint32_t pk[16];
+          for (int c = 0; c < 4; ++c) {
+            float o[32];
+            tmem_ld32(o_col + c * 32, o);
+            tmem_ld_wait32(o);
+            uint32_t pk[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            pk[e] = pack_bf16x2(o[2 * e] * inv, o[2 * e + 1] * inv);
-          if (row < args.Lq) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+            for (int e = 0; e < 16; ++e)
+              pk[e] = pack_bf16x2(o[2 * e] * inv, o[2 * e + 1] * inv);
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-              dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2],
-                                  pk[4 * e + 3]);
+            for (int e = 0; e < 4; ++e) {
+              const int cc = c * 4 + e;  // 16-byte chunk of the 256-byte row
+              *reinterpret_cast<uint4*>(stg + (cc >> 3) * HALF + r * 128 +
+                                        (((cc & 7) ^ (r & 7)) << 4)) =
+                  make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2],
+                             pk[4 * e + 3]);
+            }
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar[B_OWRITTEN + t]);
+          if ((warp & 3) == 0) {
+            const bool written =
+                wait_warp(&bar[B_OWRITTEN + t], 0, abort_flag, status);
+            if (written && lane == 0) {
+              tma_store_4d(&tm_o, stg, 0, ce.head, ce.q0 + t * BM, ce.b);
+              tma_store_4d(&tm_o, stg + HALF, 64, ce.head, ce.q0 + t * BM,
+                           ce.b);
+              bulk_commit_group();
+            }
+            __syncwarp();
           }
         }
         // O_t has been read: the next item's first P V may overwrite it
@@ -869,7 +890,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // the output stores of the staging buffers are complete before the CTA
   // (and its shared memory) goes away
-  if (kPersist && warp < 8 && (warp & 3) == 0 && lane == 0) bulk_wait_group0();
+  if (warp < 8 && (warp & 3) == 0 && lane == 0) bulk_wait_group0();
   tc_fence_before();
   __syncthreads();
   if (warp == 9) {
@@ -1523,8 +1544,11 @@ int wan_self_attn(const void* q, const void* k, const void* v, void* o,
   a.cross = 0;
   a.chunk = 0;
   a.q_offset = 0;
-  return d_table ? launch<1, 0>(mq, mk, mv, mq, a, B, as_stream(s))
-                 : launch<0, 0>(mq, mk, mv, mq, a, B, as_stream(s));
+  CUtensorMap mo;
+  if ((st = make_map_bf16(&mo, o, B, a.Lq, heads, BM)) != WAN_OK)
+    return st;
+  return d_table ? launch<1, 0>(mq, mk, mv, mo, a, B, as_stream(s))
+                 : launch<0, 0>(mq, mk, mv, mo, a, B, as_stream(s));
 }
 
 int wan_self_attn_rope_q(const void* q, const void* k, const void* v,
@@ -1560,7 +1584,10 @@ int wan_self_attn_rope_q(const void* q, const void* k, const void* v,
   a.cross = 0;
   a.chunk = 0;
   a.q_offset = 0;
-  return launch<2, 0>(mq, mk, mv, mq, a, B, as_stream(s));
+  CUtensorMap mo;
+  if ((st = make_map_bf16(&mo, o, B, a.Lq, heads, BM)) != WAN_OK)
+    return st;
+  return launch<2, 0>(mq, mk, mv, mo, a, B, as_stream(s));
 }
 
 int wan_self_attn_pair(const void* q, const void* k, const void* v, void* o,
@@ -1692,7 +1719,10 @@ int wan_block_causal_attn_split(const void* q, const void* k, const void* v,
     a.split_rows = rows;
   }
   cudaStream_t cs = as_stream(s);
-  st = launch<0, 0>(mq, mk, mv, mq, a, B, cs);
+  CUtensorMap mo;
+  if ((st = make_map_bf16(&mo, o, B, a.Lq, heads, BM)) != WAN_OK)
+    return st;
+  st = launch<0, 0>(mq, mk, mv, mo, a, B, cs);
   if (st != WAN_OK || n_split == 1) return st;
   const int64_t blocks64 = (rows + 7) / 8;
   const int blocks = static_cast<int>(blocks64 < 148 * 16 ? blocks64 : 148 * 16);
@@ -1837,7 +1867,10 @@ int wan_block_causal_attn(const void* q, const void* k, const void* v,
   a.cross = 0;
   a.chunk = chunk_tokens;
   a.q_offset = q_offset;
-  return launch<0, 0>(mq, mk, mv, mq, a, B, as_stream(s));
+  CUtensorMap mo;
+  if ((st = make_map_bf16(&mo, o, B, a.Lq, heads, BM)) != WAN_OK)
+    return st;
+  return launch<0, 0>(mq, mk, mv, mo, a, B, as_stream(s));
 }
 
 int wan_cross_attn(const void* q, const void* k_ctx, const void* v_ctx,
