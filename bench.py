@@ -213,11 +213,11 @@ def run_reference(args, w, rank, world):
 
 # DRAM bytes per algorithmic byte (Q, K, V read once, O written once) of the
 # self-attention kernel, from the ncu capture of the 480p-81f launch:
-# 797.29 MB measured (613.50 read + 183.79 written) for 805.31 MB
+# 812.18 MB measured (626.39 read + 185.78 written) for 805.31 MB
 # algorithmic.  The kernel's DRAM traffic grows in proportion to
 # B * L * heads, so a launch's traffic is this ratio times its algorithmic
 # bytes.
-ATTN_DRAM_PER_ALG_BYTE = 797.29 / 805.31
+ATTN_DRAM_PER_ALG_BYTE = 812.18 / 805.31
 
 
 def rank_seed_offset(rank):
