@@ -911,13 +911,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 // block j runs, and the softmax of one block never waits on the P V and
 // Q K^T of the previous one (the two-tile kernel above has that chain).
 //
-// Per CTA (320 threads):
-//   warps 0-7  softmax: warp w owns query rows 32 (w & 3) .. + 31 (TMEM
-//              lane quadrant w & 3) and keys 64 (w >> 2) .. + 63 of every
-//              block; the two warps of a quadrant swap row maxima through
-//              shared memory (an mbarrier per quadrant), rescale their half
-//              of O when the max grows by more than 2^8, and write P (bf16)
-//              over the scores they have read.
+// Per CTA (384 threads, registers rebalanced with setmaxnreg):
+//   warps 0-7  softmax, two warps per TMEM lane quadrant: warp w owns query
+//              rows 32 (w & 3) .. + 31 and every other key block (blocks j
+//              with j % 2 == w >> 2), all 128 keys of each.  The running row
+//              max passes from block to block through shared memory (an
+//              mbarrier per quadrant): the warp of block j posts it right
+//              after its block max, so the warp of block j+1 waits only for
+//              that, not for block j's exponentials, and the two warps of a
+//              sub-partition work on different blocks at once.  The warp
+//              whose block raises the max by more than 2^8 rescales O (after
+//              P V of the previous block); each warp keeps its own row sum
+//              relative to the max it last used.
 //   warp 8     TMA producer: this CTA's Q rows, its 64 keys of each K block
 //              (3 blocks ahead of V) and its 64 channels of each V block.
 //   warp 9     in CTA 0: the MMA issuer for the pair; in CTA 1: forwards the
@@ -926,7 +931,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 //              once, in shared memory, before any MMA reads them; K comes
 //              in already rotated.
 // Tensor memory (512 columns, both CTAs): O at 0, score slot b at 128 + 128 b;
-// P of keys 0-63 / 64-127 over score columns 0-31 / 64-95 of the slot.
+// P (bf16) of a block over the first 64 columns of its slot.
 namespace pair {
 constexpr int RM = 128;                    // query rows per CTA
 constexpr int NSLOT = 3;                   // score / P slots
@@ -938,7 +943,7 @@ constexpr uint32_t KHALF = 8192;           // [64 keys][64 ch] bf16
 constexpr uint32_t KTILE = 2 * KHALF;
 constexpr uint32_t VTILE = 16384;          // [128 keys][64 ch] bf16
 constexpr uint32_t SMEM = QTILE + KSTAGES * KTILE + VSTAGES * VTILE + 1024;
-constexpr int THREADS = 320;               // 384 with the Q-rotation warps
+constexpr int THREADS = 384;
 constexpr uint32_t TM_SLOT0 = 128;
 constexpr uint16_t BOTH = 3;               // multicast mask: CTAs 0 and 1
 constexpr uint32_t IDESC_S2 = idesc_bf16_f32(2 * RM, BN, 0);
@@ -954,19 +959,19 @@ enum : int {
   KEMPTY = VPEER + VSTAGES,       // per stage: the pair's MMAs are done with it
   VEMPTY = KEMPTY + KSTAGES,
   SFULL = VEMPTY + VSTAGES,       // per slot: S written (both CTAs)
-  PREADY = SFULL + NSLOT,     // per slot: P written by all 16 softmax warps
+  PREADY = SFULL + NSLOT,     // per slot: P written by the block's 8 warps
   PVDONE = PREADY + NSLOT,    // per slot: P V done (both CTAs)
   OFINAL = PVDONE + NSLOT,    // the item's last P V done (both CTAs)
   DRAIN = OFINAL + 1,         // every MMA done (both CTAs)
-  XCH = DRAIN + 1,            // per lane quadrant: both key halves posted
-  QREADY = XCH + 4,           // (kRopeQ) this CTA's Q rows rotated
+  XCH = DRAIN + 1,            // per lane quadrant: both row sums posted
+  MCHAIN = XCH + 4,           // per lane quadrant: a block's row max posted
+  QREADY = MCHAIN + 4,        // (kRopeQ) this CTA's Q rows rotated
   NUM_BARS = QREADY + 1
 };
 }  // namespace pair
 
 template <int kRopeQ>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(
-    pair::THREADS + 64 * kRopeQ, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::THREADS, 1)
     attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v,
@@ -976,7 +981,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(
   __shared__ __align__(8) uint64_t bar[NUM_BARS];
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
-  __shared__ float s_xch[2][2][RM];  // [block parity][key half][row]
+  __shared__ float s_xch[2][RM];     // [warp set][row]: final row sums
+  __shared__ float s_mx[2][RM];      // [block parity][row]: running max
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -1024,12 +1030,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(
     }
     for (int i = 0; i < NSLOT; ++i) {
       mbar_init(&bar[SFULL + i], 1);
-      mbar_init(&bar[PREADY + i], 16);
+      mbar_init(&bar[PREADY + i], 8);
       mbar_init(&bar[PVDONE + i], 1);
     }
     mbar_init(&bar[OFINAL], 1);
     mbar_init(&bar[DRAIN], 1);
-    for (int i = 0; i < 4; ++i) mbar_init(&bar[XCH + i], 2);
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&bar[XCH + i], 2);
+      mbar_init(&bar[MCHAIN + i], 1);
+    }
     mbar_init(&bar[QREADY], 64);
     fence_mbar_init();
   }
@@ -1041,6 +1050,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(
   tc_fence_after();
   const uint32_t tmem = s_tmem;
 
+  if (warp >= 8) setmaxnreg_dec();
   if (warp == 8) {
     // --------------------------------------------------------- producer --
     const bool el = elect_one();
@@ -1166,9 +1176,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(
       if (el) {
 #pragma unroll
         for (int k = 0; k < BN / 16; ++k) {
-          // P of keys 16k .. 16k+15: key half k >> 2 at column 64 (k >> 2)
-          umma_ts_pair(tmem, a0 + 64 * (k >> 2) + 8 * (k & 3),
-                       b0 + ((k * 2048) >> 4), IDESC_PV2,
+          // P of keys 16k .. 16k+15 in columns 8k .. 8k+7 of the slot
+          umma_ts_pair(tmem, a0 + 8 * k, b0 + ((k * 2048) >> 4), IDESC_PV2,
                        (j > 0 || k > 0) ? 1u : 0u);
         }
         umma_commit_pair(&bar[PVDONE + sl], BOTH);
@@ -1193,11 +1202,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(
     }
   } else if (warp < 8) {
     // ---------------------------------------------------------- softmax --
+    setmaxnreg_inc();
     const int qd = warp & 3;
-    const int h = warp >> 2;
+    const int h = warp >> 2;  // warp set: blocks j with j % 2 == h
     const int r = qd * 32 + lane;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(qd * 32) << 16);
-    const uint32_t o_col = lane_base + 64 * h;
     const float c2 = args.scale_log2;
     // keys this row may see: all kv_len, or its block-causal limit
     int row_lim = kv_len;
@@ -1205,73 +1214,69 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(
       const int pos = q0 + r + args.q_offset;
       row_lim = min(args.Lk, (pos / args.chunk + 1) * args.chunk);
     }
-    float m_run = -INFINITY;
-    float l_run = 0.f;
+    float m_w = -INFINITY;  // the max this warp last used
+    float l_w = 0.f;        // this warp's row sum, relative to m_w
     bool ok = true;
-    for (int j = 0; j < nblk && ok; ++j) {
+    for (int j = h; j < nblk && ok; j += 2) {
       const int sl = j % NSLOT;
       ok = wait_warp(&bar[SFULL + sl], (j / NSLOT) & 1, abort_flag, status);
       if (!ok) break;
       tc_fence_after();
-      const uint32_t s_col = lane_base + TM_SLOT0 + sl * 128 + 64 * h;
-      float s[64];
-      tmem_ld64(s_col, s);
-      tmem_ld_wait64(s);
-      const int lim = row_lim - j * BN - 64 * h;  // valid keys of this half
-      const bool masked = __any_sync(0xffffffffu, lim < 64);
+      const uint32_t s_col = lane_base + TM_SLOT0 + sl * 128;
+      float s[BN];
+      tmem_ld128(s_col, s);
+      tmem_ld_wait128(s);
+      const int lim = row_lim - j * BN;  // valid keys of this row here
+      const bool masked = __any_sync(0xffffffffu, lim < BN);
       if (masked) {
 #pragma unroll
-        for (int c = 0; c < 64; ++c)
+        for (int c = 0; c < BN; ++c)
           if (c >= lim) s[c] = -INFINITY;
       }
-      float mx = (masked ? rowmax_masked<64>(s) : rowmax<64>(s)) * c2;
-      // both key halves of the row: swap maxima with the quadrant's partner
-      s_xch[j & 1][h][r] = mx;
+      const float mx = (masked ? rowmax_masked<BN>(s) : rowmax<BN>(s)) * c2;
+      // running max after block j: the previous block's, unless this block
+      // exceeds it by more than 2^8 (p <= 256, exact after the final O / l)
+      float m_prev = -INFINITY;
+      if (j > 0) {
+        ok = wait_warp(&bar[MCHAIN + qd], (j - 1) & 1, abort_flag, status);
+        if (!ok) break;
+        m_prev = s_mx[(j - 1) & 1][r];
+      }
+      const bool need = j > 0 && mx > m_prev + RESCALE_LOG2;
+      const float m_j = (j == 0 || need) ? mx : m_prev;
+      s_mx[j & 1][r] = m_j;
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bar[XCH + qd]);
-      ok = wait_warp(&bar[XCH + qd], j & 1, abort_flag, status);
-      if (!ok) break;
-      mx = fmaxf(mx, s_xch[j & 1][h ^ 1][r]);
-      if (j == 0) {
-        m_run = mx;
-      } else {
-        // Keep the running max unless it grew by more than 2^8 (p <= 256,
-        // exact after the final O / l); otherwise rescale this warp's half
-        // of O once P V(j-1) has landed in it.  Both warps of the quadrant
-        // see the same maxima, so they take the same decision.
-        const bool need = mx > m_run + RESCALE_LOG2;
-        if (__any_sync(0xffffffffu, need)) {
-          const float m_new = need ? mx : m_run;
-          const float alpha = ex2(m_run - m_new);
-          ok = wait_warp(&bar[PVDONE + (j - 1) % NSLOT],
-                         ((j - 1) / NSLOT) & 1, abort_flag, status);
-          if (!ok) break;
-          tc_fence_after();
+      if (lane == 0) mbar_arrive(&bar[MCHAIN + qd]);
+      if (__any_sync(0xffffffffu, need)) {
+        // O holds blocks 0 .. j-1 at m_prev once P V(j-1) has landed
+        const float alpha = ex2(m_prev - m_j);
+        ok = wait_warp(&bar[PVDONE + (j - 1) % NSLOT], ((j - 1) / NSLOT) & 1,
+                       abort_flag, status);
+        if (!ok) break;
+        tc_fence_after();
 #pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            float o[32];
-            tmem_ld32(o_col + c * 32, o);
-            tmem_ld_wait32(o);
+        for (int c = 0; c < 4; ++c) {
+          float o[32];
+          tmem_ld32(lane_base + c * 32, o);
+          tmem_ld_wait32(o);
 #pragma unroll
-            for (int e = 0; e < 32; e += 2) {
-              const float2 v =
-                  ffma2(make_float2(o[e], o[e + 1]),
-                        make_float2(alpha, alpha), make_float2(0.f, 0.f));
-              o[e] = v.x;
-              o[e + 1] = v.y;
-            }
-            tmem_st32(o_col + c * 32, o);
+          for (int e = 0; e < 32; e += 2) {
+            const float2 v =
+                ffma2(make_float2(o[e], o[e + 1]), make_float2(alpha, alpha),
+                      make_float2(0.f, 0.f));
+            o[e] = v.x;
+            o[e + 1] = v.y;
           }
-          l_run *= alpha;
-          m_run = m_new;
+          tmem_st32(lane_base + c * 32, o);
         }
       }
       float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                        make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
       if (masked)
-        exp_store_chunks<false>(s, c2, m_run, s_col, acc, 0, 2);
+        exp_store_chunks<false>(s, c2, m_j, s_col, acc, 0, BN / 32);
       else
-        exp_store_chunks<true, kPairEmu8>(s, c2, m_run, s_col, acc, 0, 2);
+        exp_store_chunks<true, kPairEmu8>(s, c2, m_j, s_col, acc, 0,
+                                          BN / 32);
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -1283,23 +1288,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(
               mapa_shared(smem_u32(&bar[PREADY + sl]), 0));
       }
       const float2 tsum = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
-      l_run += tsum.x + tsum.y;
+      l_w = l_w * ex2(m_w - m_j) + (tsum.x + tsum.y);
+      m_w = m_j;
     }
+    // the final max is the last block's; both sets' sums relative to it
+    if (ok) ok = wait_warp(&bar[MCHAIN + qd], (nblk - 1) & 1, abort_flag,
+                           status);
     if (ok) ok = wait_warp(&bar[OFINAL], 0, abort_flag, status);
     if (ok) {
-      // row sum over both key halves
-      s_xch[nblk & 1][h][r] = l_run;
+      const float m_fin = s_mx[(nblk - 1) & 1][r];
+      s_xch[h][r] = m_w == -INFINITY ? 0.f : l_w * ex2(m_w - m_fin);
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar[XCH + qd]);
-      ok = wait_warp(&bar[XCH + qd], nblk & 1, abort_flag, status);
+      ok = wait_warp(&bar[XCH + qd], 0, abort_flag, status);
     }
     if (ok) {
       tc_fence_after();
-      const float inv = 1.0f / (l_run + s_xch[nblk & 1][h ^ 1][r]);
-      const int row = q0 + r;
+      const float inv = 1.0f / (s_xch[0][r] + s_xch[1][r]);
+      // the item's coordinates again, rather than held through the loop
+      int it_e = static_cast<int>(blockIdx.x >> 1);
+      asm volatile("" : "+r"(it_e));
+      const int tx_e = it_e % args.n_tiles_x;
+      const int head_e = (it_e / args.n_tiles_x) % args.heads;
+      const int b_e = it_e / args.n_tiles_x / args.heads;
+      const int tile_e = args.chunk ? args.n_tiles_x - 1 - tx_e : tx_e;
+      const int row = tile_e * (2 * RM) + static_cast<int>(rank) * RM + r;
+      const uint32_t o_col = lane_base + 64 * h;  // this set's 64 channels
       __nv_bfloat16* orow =
-          args.o + ((static_cast<int64_t>(bb) * args.Lq + row) * args.heads +
-                    head) * HD + 64 * h;
+          args.o + ((static_cast<int64_t>(b_e) * args.Lq + row) * args.heads +
+                    head_e) * HD + 64 * h;
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         float o[32];
@@ -1455,6 +1472,13 @@ int launch_pair(const CUtensorMap& mq, const CUtensorMap& mk,
   {
     std::lock_guard<std::mutex> lock(mu);
     if (state[dev] == 0) {
+      // setmaxnreg draws on the registers the CTA was launched with
+      cudaFuncAttributes fa;
+      if (cudaFuncGetAttributes(&fa, attn_pair_kernel<kRopeQ>) != cudaSuccess)
+        return WAN_ECUDA;
+      if (fa.numRegs * pair::THREADS <
+          8 * 32 * kSoftmaxRegs + 4 * 32 * kOtherRegs)
+        return WAN_EUNSUPPORTED;
       if (cudaFuncSetAttribute(attn_pair_kernel<kRopeQ>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                pair::SMEM) != cudaSuccess)
@@ -1466,9 +1490,8 @@ int launch_pair(const CUtensorMap& mq, const CUtensorMap& mk,
   const int64_t items = static_cast<int64_t>(a.n_tiles_x) * a.heads * B;
   if (2 * items > INT32_MAX) return WAN_EINVAL;
   a.items = static_cast<int>(items);
-  attn_pair_kernel<kRopeQ>
-      <<<static_cast<unsigned>(2 * items), pair::THREADS + 64 * kRopeQ,
-         pair::SMEM, s>>>(mq, mk, mv, a);
+  attn_pair_kernel<kRopeQ><<<static_cast<unsigned>(2 * items), pair::THREADS,
+                             pair::SMEM, s>>>(mq, mk, mv, a);
   return cudaGetLastError() == cudaSuccess ? WAN_OK : WAN_ECUDA;
 }
 
