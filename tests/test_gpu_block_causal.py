@@ -67,6 +67,26 @@ def test_kv_cache_chunk_step(chunk, n_chunks, pair):
     assert_attn_close(got, want, "kv-cache chunk %d" % chunk)
 
 
+def test_default_runs_the_pair_kernel():
+    # pair=None (the default) takes the CTA-pair kernel unless key ranges
+    # are asked for: bit-identical to pair=True, and with split= to the
+    # two-tile kernel's key ranges
+    L, chunk = 600, 120
+    q, k, v = _qkv(1, chunk, L, 2, 4242)
+    qg, kg, vg = cuda(q), cuda(k), cuda(v)
+    outs = {}
+    for name, kw in (("default", {}), ("pair", {"pair": True}),
+                     ("split2", {"split": 2}),
+                     ("tiles2", {"pair": False, "split": 2})):
+        o = torch.empty_like(qg)
+        wan.block_causal_attn(qg, kg, vg, o, chunk, L - chunk, **kw)
+        outs[name] = o
+    torch.cuda.synchronize()
+    assert wan.device_status() == 0
+    assert torch.equal(outs["default"], outs["pair"])
+    assert torch.equal(outs["split2"], outs["tiles2"])
+
+
 @pytest.mark.parametrize("L,chunk,q_offset,Lq,n_split", [
     (600, 120, 480, 120, 2),     # KV-cache step, equal items
     (600, 120, 480, 120, 3),
