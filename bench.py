@@ -392,8 +392,10 @@ def causal_rooflines(dev, peak_tflops, reps=5):
     52 = 65,520 tokens, 40 heads, chunks of 3 latent frames (4,680 tokens).
     Times the full-sequence call and the KV-cache step of the last chunk
     (4,680 queries against all 65,520 keys) as the binding runs them by
-    default (the CTA-pair kernel), and beside them the two-tile kernel: the
-    full sequence, and the KV-cache step with the key ranges
+    default (block_causal_default_pair: the two-tile kernel for the full
+    sequence, the CTA-pair kernel for the KV-cache step), and beside them
+    the other kernel: the full sequence on the CTA-pair kernel, the
+    KV-cache step on the two-tile kernel with the key ranges
     wan_block_causal_attn_splits picks (plus the combining pass) and with
     one range.  The calls are timed in turn, one launch of each per round,
     and each reports its median.  FLOPs count only visible keys:
@@ -425,21 +427,21 @@ def causal_rooflines(dev, peak_tflops, reps=5):
     n_split = wan.block_causal_splits(1, chunk, L, H, chunk, L - chunk)
     ws = torch.empty(max(1, wan.block_causal_workspace_bytes(
         1, chunk, H, n_split)), dtype=torch.uint8, device=dev)
-    # (name, queries, offset, pair kernel, key ranges): the first two are
-    # the binding's default (pair=None: the CTA-pair kernel), the rest the
-    # two-tile kernel
-    cases = (("full_sequence", q, 0, True, 1),
-             ("kv_cache_last_chunk", ql, L - chunk, True, 1),
-             ("full_sequence_two_tile", q, 0, False, 1),
-             ("kv_cache_last_chunk_key_ranges", ql, L - chunk, False, n_split),
-             ("kv_cache_last_chunk_one_range", ql, L - chunk, False, 1))
+    # (name, queries, offset, pair kernel or None for the binding's
+    # default, key ranges)
+    cases = (("full_sequence", q, 0, None, 1),
+             ("kv_cache_last_chunk", ql, L - chunk, None, 1),
+             ("full_sequence_pair", q, 0, True, 1),
+             ("kv_cache_last_chunk_two_tile_key_ranges", ql, L - chunk,
+              False, n_split),
+             ("kv_cache_last_chunk_two_tile_one_range", ql, L - chunk, False,
+              1))
     calls = []
     for name, qq, off, pair, sp in cases:
         oo = o[:, :qq.shape[1]] if off else o
 
         def call(qq=qq, oo=oo, off=off, pair=pair, sp=sp):
-            wan.block_causal_attn(qq, k, v, oo, chunk, off,
-                                  pair=None if pair else False,
+            wan.block_causal_attn(qq, k, v, oo, chunk, off, pair=pair,
                                   split=sp if sp > 1 else None,
                                   workspace=ws if sp > 1 else None)
         for _ in range(2):
@@ -457,6 +459,9 @@ def causal_rooflines(dev, peak_tflops, reps=5):
             torch.cuda.synchronize()
             times[i].append(e0.elapsed_time(e1))
     for (name, qq, off, pair, sp), t in zip(cases, times):
+        if pair is None:
+            pair = wan.block_causal_default_pair(1, qq.shape[1], L, H, chunk,
+                                                 off)
         ms = float(np.median(t))
         fl = 4.0 * 128 * H * visible(qq.shape[1], off)
         out[name] = {"ms": ms, "tflops": fl / (ms / 1e3) / 1e12,

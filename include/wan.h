@@ -254,6 +254,29 @@ int wan_block_causal_attn_pair(const void* q, const void* k, const void* v,
                                int head_dim, int chunk_tokens, int q_offset,
                                float softmax_scale, void* s);
 
+/* wan_block_causal_attn_split on the CTA-pair kernel: each (256-row tile,
+ * head, batch row) pair item's key blocks cut into n_split consecutive
+ * ranges run as separate CTA pairs, then the same combining pass.  The
+ * workspace has the size and layout of wan_block_causal_attn_split's
+ * (wan_block_causal_attn_workspace_bytes); arguments, errors and results
+ * are those of wan_block_causal_attn_split.                                */
+int wan_block_causal_attn_pair_split(const void* q, const void* k,
+                                     const void* v, void* o, int B, int Lq,
+                                     int Lk, int heads, int head_dim,
+                                     int chunk_tokens, int q_offset,
+                                     float softmax_scale, int n_split,
+                                     void* workspace, size_t workspace_bytes,
+                                     void* s);
+
+/* Key-range count for wan_block_causal_attn_pair_split: 1 unless every
+ * item sees the same keys; otherwise the count up to 4 (at least 8 key
+ * blocks a range) whose waves of CTA pairs on the current device
+ * (wan_attn_pair_resident_clusters) are fullest once a split count's fill
+ * is discounted by 6 %, the measured cost of the partials and the
+ * combining pass.  Returns a negative wan_status on failure.              */
+int wan_block_causal_attn_pair_splits(int B, int Lq, int Lk, int heads,
+                                      int chunk_tokens, int q_offset);
+
 /* How many CTA pairs of the pair kernels can be resident at once on the
  * current device (clusters of two CTAs must share a GPC, so an SM left over
  * in a GPC with an odd number of SMs runs none).  A diagnostic; returns a

@@ -187,27 +187,25 @@ def test_split_block_causal_host_checks(lib):
     ws = ctypes.c_void_p(1 << 24)
     need = lib.wan_block_causal_attn_workspace_bytes(1, 600, 2, 2)
     L = lib
-    # n_split out of range
-    assert L.wan_block_causal_attn_split(p, p, p, o, 1, 600, 600, 2, 128,
-                                         120, 0, 0.1, 0, ws, need, None) \
-        == wan.WAN_EINVAL
-    assert L.wan_block_causal_attn_split(p, p, p, o, 1, 600, 600, 2, 128,
-                                         120, 0, 0.1, 9, ws, need, None) \
-        == wan.WAN_EINVAL
-    # the lightest item (the first 256 queries, keys < 256) has 2 key
-    # blocks: 3 ranges would leave one empty
-    assert L.wan_block_causal_attn_split(p, p, p, o, 1, 600, 600, 2, 128,
-                                         128, 0, 0.1, 3, ws, 1 << 20, None) \
-        == wan.WAN_EINVAL
-    # workspace missing, too small, misaligned
-    assert L.wan_block_causal_attn_split(p, p, p, o, 1, 600, 600, 2, 128,
-                                         120, 0, 0.1, 2, None, need, None) \
-        == wan.WAN_EINVAL
-    assert L.wan_block_causal_attn_split(p, p, p, o, 1, 600, 600, 2, 128,
-                                         120, 0, 0.1, 2, ws, need - 1, None) \
-        == wan.WAN_EINVAL
-    assert L.wan_block_causal_attn_split(p, p, p, o, 1, 600, 600, 2, 128,
-                                         120, 0, 0.1, 2,
-                                         ctypes.c_void_p((1 << 24) + 8),
-                                         need, None) == wan.WAN_EALIGN
+    for fn in (L.wan_block_causal_attn_split,
+               L.wan_block_causal_attn_pair_split):
+        # n_split out of range
+        assert fn(p, p, p, o, 1, 600, 600, 2, 128, 120, 0, 0.1, 0, ws, need,
+                  None) == wan.WAN_EINVAL
+        assert fn(p, p, p, o, 1, 600, 600, 2, 128, 120, 0, 0.1, 9, ws, need,
+                  None) == wan.WAN_EINVAL
+        # the lightest item (the first 256 queries, keys < 256) has 2 key
+        # blocks: 3 ranges would leave one empty
+        assert fn(p, p, p, o, 1, 600, 600, 2, 128, 128, 0, 0.1, 3, ws,
+                  1 << 20, None) == wan.WAN_EINVAL
+        # workspace missing, too small, misaligned
+        assert fn(p, p, p, o, 1, 600, 600, 2, 128, 120, 0, 0.1, 2, None,
+                  need, None) == wan.WAN_EINVAL
+        assert fn(p, p, p, o, 1, 600, 600, 2, 128, 120, 0, 0.1, 2, ws,
+                  need - 1, None) == wan.WAN_EINVAL
+        assert fn(p, p, p, o, 1, 600, 600, 2, 128, 120, 0, 0.1, 2,
+                  ctypes.c_void_p((1 << 24) + 8), need, None) \
+            == wan.WAN_EALIGN
     assert L.wan_block_causal_attn_splits(1, 10, 5, 2, 4, 0) == wan.WAN_EINVAL
+    assert L.wan_block_causal_attn_pair_splits(1, 10, 5, 2, 4, 0) \
+        == wan.WAN_EINVAL

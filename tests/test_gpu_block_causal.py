@@ -67,24 +67,30 @@ def test_kv_cache_chunk_step(chunk, n_chunks, pair):
     assert_attn_close(got, want, "kv-cache chunk %d" % chunk)
 
 
-def test_default_runs_the_pair_kernel():
-    # pair=None (the default) takes the CTA-pair kernel unless key ranges
-    # are asked for: bit-identical to pair=True, and with split= to the
-    # two-tile kernel's key ranges
-    L, chunk = 600, 120
-    q, k, v = _qkv(1, chunk, L, 2, 4242)
+@pytest.mark.parametrize("Lq,Lk,chunk,expect_pair", [
+    (256, 4096, 256, True),    # KV-cache step: equal items, the two-tile
+                               # kernel would cut them into key ranges
+    (600, 600, 120, False),    # full sequence: unequal items
+])
+def test_default_kernel(Lq, Lk, chunk, expect_pair):
+    # pair=None (the default) runs the kernel block_causal_default_pair
+    # names: bit-identical to asking for it
+    off = Lk - Lq
+    assert wan.block_causal_default_pair(1, Lq, Lk, 2, chunk, off) \
+        == expect_pair
+    q, k, v = _qkv(1, Lq, Lk, 2, 4242 + Lk)
     qg, kg, vg = cuda(q), cuda(k), cuda(v)
     outs = {}
-    for name, kw in (("default", {}), ("pair", {"pair": True}),
+    for name, kw in (("default", {}), ("named", {"pair": expect_pair}),
                      ("split2", {"split": 2}),
-                     ("tiles2", {"pair": False, "split": 2})):
+                     ("named2", {"pair": expect_pair, "split": 2})):
         o = torch.empty_like(qg)
-        wan.block_causal_attn(qg, kg, vg, o, chunk, L - chunk, **kw)
+        wan.block_causal_attn(qg, kg, vg, o, chunk, off, **kw)
         outs[name] = o
     torch.cuda.synchronize()
     assert wan.device_status() == 0
-    assert torch.equal(outs["default"], outs["pair"])
-    assert torch.equal(outs["split2"], outs["tiles2"])
+    assert torch.equal(outs["default"], outs["named"])
+    assert torch.equal(outs["split2"], outs["named2"])
 
 
 @pytest.mark.parametrize("L,chunk,q_offset,Lq,n_split", [
@@ -95,7 +101,8 @@ def test_default_runs_the_pair_kernel():
                                  # the second range (row max stays -inf)
     (520, 200, 0, 520, 2),       # chunk boundaries mid-block
 ])
-def test_split_key_ranges(L, chunk, q_offset, Lq, n_split):
+@pytest.mark.parametrize("pair", [False, True], ids=["tiles", "pair"])
+def test_split_key_ranges(L, chunk, q_offset, Lq, n_split, pair):
     q, k, v = _qkv(2, L, L, 2, 1300 + L + n_split)
     ql = q[:, q_offset:q_offset + Lq].contiguous()
     qg, kg, vg = cuda(ql), cuda(k), cuda(v)
@@ -103,7 +110,7 @@ def test_split_key_ranges(L, chunk, q_offset, Lq, n_split):
     ws = torch.full((wan.block_causal_workspace_bytes(2, Lq, 2, n_split),),
                     255, dtype=torch.uint8, device="cuda")  # NaN-patterned
     wan.block_causal_attn(qg, kg, vg, o, chunk, q_offset, split=n_split,
-                          workspace=ws)
+                          workspace=ws, pair=pair)
     torch.cuda.synchronize()
     assert wan.device_status() == 0
     check_guards(buf, guard)
@@ -190,17 +197,23 @@ def test_kv_cache_last_chunk_480p_165f_sampled(pair):
     _per_head(got, ql, k, v, rows, q0, "480p-165f KV step")
 
 
-def test_kv_cache_last_chunk_480p_165f_split_sampled():
-    # the launch bench.py times: key ranges chosen for this device (3 on
-    # 148 SMs: 760 equal items would fill 5.1 waves), combining pass after
+@pytest.mark.parametrize("pair", [False, True], ids=["tiles", "pair"])
+def test_kv_cache_last_chunk_480p_165f_split_sampled(pair):
+    # two-tile kernel: the key ranges its policy picks for this device (3 on
+    # 148 SMs, as 760 equal items would fill 5.1 waves); CTA-pair kernel:
+    # 2 ranges (its policy keeps one here, as splitting measured slower);
+    # combining pass after
     q, k, v = _full_qkv()
     q0 = FULL_L - FULL_CHUNK
     ql = q[:, q0:].contiguous()
-    n = wan.block_causal_splits(1, FULL_CHUNK, FULL_L, FULL_H, FULL_CHUNK, q0)
+    n = wan.block_causal_splits(1, FULL_CHUNK, FULL_L, FULL_H, FULL_CHUNK, q0,
+                                pair=pair)
+    if pair:
+        n = 2
     assert n > 1
     qg, kg, vg = cuda(ql), cuda(k), cuda(v)
     o = torch.empty_like(qg)
-    wan.block_causal_attn(qg, kg, vg, o, FULL_CHUNK, q0, split="auto")
+    wan.block_causal_attn(qg, kg, vg, o, FULL_CHUNK, q0, split=n, pair=pair)
     torch.cuda.synchronize()
     assert wan.device_status() == 0
     got = f64(o)

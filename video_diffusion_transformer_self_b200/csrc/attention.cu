@@ -998,9 +998,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::THREADS, 1)
   uint8_t* sK = sm + QTILE;
   uint8_t* sV = sK + KSTAGES * KTILE;
 
-  // Work item of the pair: 256 query rows of one (head, batch row); the
-  // block-causal mode runs the tiles of a head heaviest first.
-  const int item = static_cast<int>(blockIdx.x >> 1);
+  // Work item of the pair: 256 query rows of one (head, batch row) and, with
+  // n_split > 1, one of n_split consecutive ranges of their key blocks
+  // (numbered key range fastest); the block-causal mode runs the tiles of a
+  // head heaviest first.
+  const int split = static_cast<int>(blockIdx.x >> 1) % args.n_split;
+  const int item = static_cast<int>(blockIdx.x >> 1) / args.n_split;
   const int tx = item % args.n_tiles_x;
   const int head = (item / args.n_tiles_x) % args.heads;
   const int bb = item / args.n_tiles_x / args.heads;
@@ -1012,7 +1015,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::THREADS, 1)
     const int last = min(tile * (2 * RM) + 2 * RM, args.Lq) - 1 + args.q_offset;
     kv_len = min(args.Lk, (last / args.chunk + 1) * args.chunk);
   }
-  const int nblk = (kv_len + BN - 1) / BN;
+  // this range's key blocks: kb0 .. kb0 + nblk - 1 (j below counts from 0)
+  const int nb_all = (kv_len + BN - 1) / BN;
+  const int kb0 = split * nb_all / args.n_split;
+  const int nblk = (split + 1) * nb_all / args.n_split - kb0;
 
   if (threadIdx.x == 0) {
     s_abort = 0;
@@ -1075,7 +1081,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::THREADS, 1)
                          abort_flag, status);
         if (!ok) break;
         if (el) {
-          const int key0 = j * BN + static_cast<int>(rank) * 64;
+          const int key0 = (kb0 + j) * BN + static_cast<int>(rank) * 64;
           mbar_expect_tx(&bar[KFULL + sk], KTILE);
           tma_load_4d(sK + sk * KTILE, &tm_k, &bar[KFULL + sk], 0, head, key0,
                       bb);
@@ -1095,7 +1101,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::THREADS, 1)
         if (el) {
           mbar_expect_tx(&bar[VFULL + sv], VTILE);
           tma_load_4d(sV + sv * VTILE, &tm_v, &bar[VFULL + sv],
-                      static_cast<int>(rank) * 64, head, jv * BN, bb);
+                      static_cast<int>(rank) * 64, head, (kb0 + jv) * BN,
+                      bb);
         }
         __syncwarp();
         ++nv;
@@ -1226,7 +1233,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::THREADS, 1)
       float s[BN];
       tmem_ld128(s_col, s);
       tmem_ld_wait128(s);
-      const int lim = row_lim - j * BN;  // valid keys of this row here
+      const int lim = row_lim - (kb0 + j) * BN;  // valid keys of this row
       const bool masked = __any_sync(0xffffffffu, lim < BN);
       if (masked) {
 #pragma unroll
@@ -1272,8 +1279,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::THREADS, 1)
       }
       float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                        make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+      // A row with no visible key yet (possible in a later key range) keeps
+      // m = -inf: its scores are all -inf and exponentiate against 0 to
+      // exact zeros.
       if (masked)
-        exp_store_chunks<false>(s, c2, m_j, s_col, acc, 0, BN / 32);
+        exp_store_chunks<false>(s, c2, m_j == -INFINITY ? 0.f : m_j, s_col,
+                                acc, 0, BN / 32);
       else
         exp_store_chunks<true, kPairEmu8>(s, c2, m_j, s_col, acc, 0,
                                           BN / 32);
@@ -1288,15 +1299,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::THREADS, 1)
               mapa_shared(smem_u32(&bar[PREADY + sl]), 0));
       }
       const float2 tsum = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
-      l_w = l_w * ex2(m_w - m_j) + (tsum.x + tsum.y);
+      l_w = (m_w == m_j ? l_w : l_w * ex2(m_w - m_j)) + (tsum.x + tsum.y);
       m_w = m_j;
     }
     // the final max is the last block's; both sets' sums relative to it
     if (ok) ok = wait_warp(&bar[MCHAIN + qd], (nblk - 1) & 1, abort_flag,
                            status);
     if (ok) ok = wait_warp(&bar[OFINAL], 0, abort_flag, status);
+    float m_fin = -INFINITY;
     if (ok) {
-      const float m_fin = s_mx[(nblk - 1) & 1][r];
+      m_fin = s_mx[(nblk - 1) & 1][r];
       s_xch[h][r] = m_w == -INFINITY ? 0.f : l_w * ex2(m_w - m_fin);
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar[XCH + qd]);
@@ -1304,34 +1316,59 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::THREADS, 1)
     }
     if (ok) {
       tc_fence_after();
-      const float inv = 1.0f / (s_xch[0][r] + s_xch[1][r]);
+      const float l_tot = s_xch[0][r] + s_xch[1][r];
       // the item's coordinates again, rather than held through the loop
       int it_e = static_cast<int>(blockIdx.x >> 1);
       asm volatile("" : "+r"(it_e));
+      const int split_e = it_e % args.n_split;
+      it_e /= args.n_split;
       const int tx_e = it_e % args.n_tiles_x;
       const int head_e = (it_e / args.n_tiles_x) % args.heads;
       const int b_e = it_e / args.n_tiles_x / args.heads;
       const int tile_e = args.chunk ? args.n_tiles_x - 1 - tx_e : tx_e;
       const int row = tile_e * (2 * RM) + static_cast<int>(rank) * RM + r;
       const uint32_t o_col = lane_base + 64 * h;  // this set's 64 channels
-      __nv_bfloat16* orow =
-          args.o + ((static_cast<int64_t>(b_e) * args.Lq + row) * args.heads +
-                    head_e) * HD + 64 * h;
+      const int64_t orow_i =
+          (static_cast<int64_t>(b_e) * args.Lq + row) * args.heads + head_e;
+      if (args.n_split > 1) {
+        // one key range of the row: unnormalised O (this set's channels)
+        // and (row max, row sum) for the combining pass
+        const int64_t prow = split_e * args.split_rows + orow_i;
+        float4* dst =
+            reinterpret_cast<float4*>(args.part_o + prow * HD + 64 * h);
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        float o[32];
-        tmem_ld32(o_col + c * 32, o);
-        tmem_ld_wait32(o);
-        uint32_t pk[16];
+        for (int c = 0; c < 2; ++c) {
+          float o[32];
+          tmem_ld32(o_col + c * 32, o);
+          tmem_ld_wait32(o);
+          if (row < args.Lq) {
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          pk[e] = pack_bf16x2(o[2 * e] * inv, o[2 * e + 1] * inv);
-        if (row < args.Lq) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+            for (int e = 0; e < 8; ++e)
+              dst[c * 8 + e] = make_float4(o[4 * e], o[4 * e + 1],
+                                           o[4 * e + 2], o[4 * e + 3]);
+          }
+        }
+        if (h == 0 && row < args.Lq)
+          args.part_ml[prow] = make_float2(m_fin, l_tot);
+      } else {
+        const float inv = 1.0f / l_tot;
+        __nv_bfloat16* orow = args.o + orow_i * HD + 64 * h;
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2],
-                                pk[4 * e + 3]);
+        for (int c = 0; c < 2; ++c) {
+          float o[32];
+          tmem_ld32(o_col + c * 32, o);
+          tmem_ld_wait32(o);
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            pk[e] = pack_bf16x2(o[2 * e] * inv, o[2 * e + 1] * inv);
+          if (row < args.Lq) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2],
+                                  pk[4 * e + 3]);
+          }
         }
       }
     }
@@ -1487,7 +1524,8 @@ int launch_pair(const CUtensorMap& mq, const CUtensorMap& mk,
     }
   }
   a.n_tiles_x = (a.Lq + 2 * pair::RM - 1) / (2 * pair::RM);
-  const int64_t items = static_cast<int64_t>(a.n_tiles_x) * a.heads * B;
+  const int64_t items =
+      static_cast<int64_t>(a.n_tiles_x) * a.heads * B * a.n_split;
   if (2 * items > INT32_MAX) return WAN_EINVAL;
   a.items = static_cast<int>(items);
   attn_pair_kernel<kRopeQ><<<static_cast<unsigned>(2 * items), pair::THREADS,
@@ -1515,6 +1553,39 @@ int check_common(const void* q, const void* k, const void* v, void* o, int B,
 int causal_item_kv(int tile, int Lq, int Lk, int chunk, int q_offset) {
   const int last = min((tile + 1) * QT * BM, Lq) - 1 + q_offset;
   return min(Lk, (last / chunk + 1) * chunk);
+}
+
+// Key ranges for `items` equal work items of nblk key blocks on `slots`
+// concurrent CTAs (or CTA pairs): the smallest count up to 4, with at least
+// 8 key blocks a range, whose waves are at least 95 % full (else the
+// fullest).  range_cost discounts a split count's wave fill by the
+// measured cost of its fp32 partials and combining pass.
+int split_count(double items, int nblk, int slots, double range_cost) {
+  int best = 1;
+  double best_eff = 0.0;
+  for (int sp = 1; sp <= 4; ++sp) {
+    if (sp > 1 && nblk < 8 * sp) break;  // at least 8 key blocks per range
+    const double waves = items * sp / slots;
+    const double eff = waves / ceil(waves) * (sp > 1 ? 1.0 - range_cost : 1.0);
+    if (eff > best_eff + 0.01) {
+      best = sp;
+      best_eff = eff;
+    }
+    if (eff >= 0.95) break;
+  }
+  return best;
+}
+
+// Rows of partial results and the combining pass of a split call.
+int combine_splits(const AttnArgs& a, int64_t rows, int n_split,
+                   cudaStream_t cs) {
+  const int64_t blocks64 = (rows + 7) / 8;
+  const int blocks =
+      static_cast<int>(blocks64 < 148 * 16 ? blocks64 : 148 * 16);
+  combine_splits_kernel<<<blocks, 256, 0, cs>>>(
+      reinterpret_cast<const float4*>(a.part_o), a.part_ml, a.o, rows,
+      n_split);
+  return cudaGetLastError() == cudaSuccess ? WAN_OK : WAN_ECUDA;
 }
 
 int causal_check(const void* q, const void* k, const void* v, void* o, int B,
@@ -1681,20 +1752,7 @@ int wan_block_causal_attn_splits(int B, int Lq, int Lk, int heads,
   // leaves the last wave of CTAs partly empty.
   if (kv_first != kv_last) return 1;
   const int nblk = (kv_first + BN - 1) / BN;
-  const double items = static_cast<double>(tiles) * heads * B;
-  int best = 1;
-  double best_eff = 0.0;
-  for (int sp = 1; sp <= 4; ++sp) {
-    if (sp > 1 && nblk < 8 * sp) break;  // at least 8 key blocks per range
-    const double waves = items * sp / sms;
-    const double eff = waves / ceil(waves);
-    if (eff > best_eff + 0.01) {
-      best = sp;
-      best_eff = eff;
-    }
-    if (eff >= 0.95) break;
-  }
-  return best;
+  return split_count(static_cast<double>(tiles) * heads * B, nblk, sms, 0.0);
 }
 
 int wan_block_causal_attn_split(const void* q, const void* k, const void* v,
@@ -1747,12 +1805,7 @@ int wan_block_causal_attn_split(const void* q, const void* k, const void* v,
     return st;
   st = launch<0, 0>(mq, mk, mv, mo, a, B, cs);
   if (st != WAN_OK || n_split == 1) return st;
-  const int64_t blocks64 = (rows + 7) / 8;
-  const int blocks = static_cast<int>(blocks64 < 148 * 16 ? blocks64 : 148 * 16);
-  combine_splits_kernel<<<blocks, 256, 0, cs>>>(
-      reinterpret_cast<const float4*>(a.part_o), a.part_ml, a.o, rows,
-      n_split);
-  return cudaGetLastError() == cudaSuccess ? WAN_OK : WAN_ECUDA;
+  return combine_splits(a, rows, n_split, cs);
 }
 
 // ------------------------------------------------- without allocation --
@@ -1860,6 +1913,79 @@ int wan_block_causal_attn_pair(const void* q, const void* k, const void* v,
   a.chunk = chunk_tokens;
   a.q_offset = q_offset;
   return launch_pair<0>(mq, mk, mv, a, B, as_stream(s));
+}
+
+int wan_block_causal_attn_pair_splits(int B, int Lq, int Lk, int heads,
+                                      int chunk_tokens, int q_offset) {
+  using namespace wan;
+  if (B < 1 || Lq < 1 || Lk < 1 || heads < 1 || chunk_tokens < 1 ||
+      q_offset < 0 || static_cast<int64_t>(q_offset) + Lq > Lk)
+    return WAN_EINVAL;
+  const int pairs = wan_attn_pair_resident_clusters();
+  if (pairs < 1) return pairs < 0 ? pairs : WAN_EUNSUPPORTED;
+  // pair items hold 256 query rows, as the two-tile kernel's do
+  const int tiles = (Lq + 2 * pair::RM - 1) / (2 * pair::RM);
+  const int kv_first = causal_item_kv(0, Lq, Lk, chunk_tokens, q_offset);
+  const int kv_last =
+      causal_item_kv(tiles - 1, Lq, Lk, chunk_tokens, q_offset);
+  if (kv_first != kv_last) return 1;
+  const int nblk = (kv_first + BN - 1) / BN;
+  // Measured at the 480p-165f KV-cache step (760 pair items on 74 pairs):
+  // 2 ranges (waves 97.8 % full) ran 1.3 % slower than one (93.4 %), so a
+  // split must buy more than about 6 % of wave fill.
+  return split_count(static_cast<double>(tiles) * heads * B, nblk, pairs,
+                     0.06);
+}
+
+int wan_block_causal_attn_pair_split(const void* q, const void* k,
+                                     const void* v, void* o, int B, int Lq,
+                                     int Lk, int heads, int head_dim,
+                                     int chunk_tokens, int q_offset,
+                                     float softmax_scale, int n_split,
+                                     void* workspace, size_t workspace_bytes,
+                                     void* s) {
+  using namespace wan;
+  int st = causal_check(q, k, v, o, B, Lq, Lk, heads, head_dim, chunk_tokens,
+                        q_offset, softmax_scale);
+  if (st != WAN_OK) return st;
+  if (n_split < 1 || n_split > 8) return WAN_EINVAL;
+  if (n_split > 1) {
+    // every key range of every item holds at least one key block
+    const int kv0 = causal_item_kv(0, Lq, Lk, chunk_tokens, q_offset);
+    if ((kv0 + BN - 1) / BN < n_split) return WAN_EINVAL;
+    const size_t need =
+        wan_block_causal_attn_workspace_bytes(B, Lq, heads, n_split);
+    if (!workspace || workspace_bytes < need) return WAN_EINVAL;
+    if (!aligned16(workspace)) return WAN_EALIGN;
+  }
+  st = check_device(nullptr);
+  if (st != WAN_OK) return st;
+  CUtensorMap mq, mk, mv;
+  if ((st = make_map_bf16(&mq, q, B, Lq, heads, 128)) != WAN_OK) return st;
+  if ((st = make_map_bf16(&mk, k, B, Lk, heads, 64)) != WAN_OK) return st;
+  if ((st = make_map_bf16(&mv, v, B, Lk, heads, 128)) != WAN_OK) return st;
+  AttnArgs a;
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.table = nullptr;
+  a.Lq = Lq;
+  a.Lk = Lk;
+  a.heads = heads;
+  a.F = a.H = a.W = 1;
+  a.scale_log2 = softmax_scale * 1.4426950408889634f;
+  a.cross = 0;
+  a.chunk = chunk_tokens;
+  a.q_offset = q_offset;
+  a.n_split = n_split;
+  const int64_t rows = static_cast<int64_t>(B) * Lq * heads;
+  if (n_split > 1) {
+    a.part_o = static_cast<float*>(workspace);
+    a.part_ml = reinterpret_cast<float2*>(a.part_o + n_split * rows * HD);
+    a.split_rows = rows;
+  }
+  cudaStream_t cs = as_stream(s);
+  st = launch_pair<0>(mq, mk, mv, a, B, cs);
+  if (st != WAN_OK || n_split == 1) return st;
+  return combine_splits(a, rows, n_split, cs);
 }
 
 int wan_block_causal_attn(const void* q, const void* k, const void* v,

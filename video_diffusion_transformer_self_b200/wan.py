@@ -84,6 +84,10 @@ _SIGNATURES = {
     "wan_block_causal_attn_workspace_bytes": (ctypes.c_size_t,
                                               [_I, _I, _I, _I]),
     "wan_block_causal_attn_splits": (_I, [_I, _I, _I, _I, _I, _I]),
+    "wan_block_causal_attn_pair_split": (_I, [_P, _P, _P, _P, _I, _I, _I,
+                                              _I, _I, _I, _I, ctypes.c_float,
+                                              _I, _P, ctypes.c_size_t, _P]),
+    "wan_block_causal_attn_pair_splits": (_I, [_I, _I, _I, _I, _I, _I]),
     "wan_block_causal_attn_split_noalloc": (_I, [_P, _P, _P, _P, _I, _I, _I,
                                                  _I, _I, _I, _I,
                                                  ctypes.c_float, _I, _P]),
@@ -363,16 +367,13 @@ def block_causal_attn(q, k, v, o, chunk_tokens, q_offset=0,
     j < (a // chunk_tokens + 1) * chunk_tokens (and j < Lk).
 
     pair: True runs the CTA-pair kernel (wan_block_causal_attn_pair), False
-    the two-tile kernel (wan_block_causal_attn); None picks the pair kernel
-    unless key ranges are asked for.  Measured at 480p-165f (65,520 tokens,
-    40 heads, 4,680-token chunks) in an interleaved A/B: the pair kernel
-    runs the KV-cache step of the last chunk 7.6 % faster than the two-tile
-    kernel with its best key ranges, and the full sequence at parity.
-    split: None (one key range per item), "auto"
-    (wan_block_causal_attn_splits) or a count, two-tile kernel only; with
-    more than one range the call needs a workspace (a CUDA tensor of at
-    least block_causal_workspace_bytes(...) bytes), allocated here with
-    torch if not given."""
+    the two-tile kernel (wan_block_causal_attn), None (the default) the
+    kernel block_causal_default_pair picks.
+    split: None (one key range per item), "auto" (block_causal_splits for
+    the kernel chosen) or a count; with more than one range the call
+    (wan_block_causal_attn_split or _pair_split) needs a workspace (a CUDA
+    tensor of at least block_causal_workspace_bytes(...) bytes), allocated
+    here with torch if not given."""
     for name, t in (("q", q), ("k", k), ("v", v), ("o", o)):
         _bf16_bl(t, name)
     B, Lq, H, D = q.shape
@@ -383,16 +384,16 @@ def block_causal_attn(q, k, v, o, chunk_tokens, q_offset=0,
     _on_cuda(("q", q), ("k", k), ("v", v), ("o", o))
     if softmax_scale is None:
         softmax_scale = 1.0 / math.sqrt(D)
+    if pair is None:
+        pair = block_causal_default_pair(B, Lq, Lk, H, chunk_tokens,
+                                         q_offset)
     n_split = 1
     if split == "auto":
-        n_split = block_causal_splits(B, Lq, Lk, H, chunk_tokens, q_offset)
+        n_split = block_causal_splits(B, Lq, Lk, H, chunk_tokens, q_offset,
+                                      pair=pair)
     elif split is not None:
         n_split = int(split)
-    if pair is None:
-        pair = split is None
     if n_split > 1:
-        if pair:
-            raise ValueError("key ranges run on the two-tile kernel only")
         need = block_causal_workspace_bytes(B, Lq, H, n_split)
         if workspace is None:
             import torch
@@ -402,11 +403,13 @@ def block_causal_attn(q, k, v, o, chunk_tokens, q_offset=0,
             raise ValueError("workspace must be a contiguous tensor of at "
                              "least %d bytes" % need)
         _on_cuda(("q", q), ("workspace", workspace))
-        _check(lib().wan_block_causal_attn_split(
+        name = "wan_block_causal_attn_pair_split" if pair else \
+            "wan_block_causal_attn_split"
+        _check(getattr(lib(), name)(
             _ptr(q), _ptr(k), _ptr(v), _ptr(o), B, Lq, Lk, H, D,
             int(chunk_tokens), int(q_offset), softmax_scale, n_split,
             _ptr(workspace), workspace.numel() * workspace.element_size(),
-            _stream(stream)), "wan_block_causal_attn_split")
+            _stream(stream)), name)
         return
     fn = lib().wan_block_causal_attn_pair if pair else \
         lib().wan_block_causal_attn
@@ -415,17 +418,34 @@ def block_causal_attn(q, k, v, o, chunk_tokens, q_offset=0,
               _stream(stream)), "wan_block_causal_attn")
 
 
+def block_causal_default_pair(B, Lq, Lk, heads, chunk_tokens, q_offset=0):
+    """The kernel block_causal_attn runs by default: the CTA-pair kernel
+    where the two-tile kernel would cut its equal work items into key
+    ranges (wan_block_causal_attn_splits > 1, e.g. a KV-cache step), the
+    two-tile kernel otherwise.  Measured at 480p-165f (65,520 tokens, 40
+    heads, 4,680-token chunks), interleaved timings on four boxes: the
+    KV-cache step of the last chunk ran -2 to +8 % (mean +4 %) on the pair
+    kernel against the two-tile kernel with its key ranges; the full
+    sequence -5 to +5 % (mean -1 %)."""
+    return block_causal_splits(B, Lq, Lk, heads, chunk_tokens, q_offset) > 1
+
+
 def block_causal_workspace_bytes(B, Lq, heads, n_split):
     """Workspace bytes of the split block-causal call."""
     return lib().wan_block_causal_attn_workspace_bytes(B, Lq, heads, n_split)
 
 
-def block_causal_splits(B, Lq, Lk, heads, chunk_tokens, q_offset=0):
-    """Key-range count the split block-causal call is fastest with."""
-    n = lib().wan_block_causal_attn_splits(B, Lq, Lk, heads,
-                                           int(chunk_tokens), int(q_offset))
+def block_causal_splits(B, Lq, Lk, heads, chunk_tokens, q_offset=0,
+                        pair=False):
+    """Key-range count for the split block-causal call on the two-tile
+    kernel (wan_block_causal_attn_splits) or, with pair=True, on the
+    CTA-pair kernel (wan_block_causal_attn_pair_splits)."""
+    name = "wan_block_causal_attn_pair_splits" if pair else \
+        "wan_block_causal_attn_splits"
+    n = getattr(lib(), name)(B, Lq, Lk, heads, int(chunk_tokens),
+                             int(q_offset))
     if n < 1:
-        _check(n, "wan_block_causal_attn_splits")
+        _check(n, name)
     return n
 
 
