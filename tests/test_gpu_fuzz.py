@@ -175,3 +175,46 @@ def test_block_causal_random(B, Lq, Lk, heads, chunk, q_offset, pair,
                                         chunk, q_offset)
     assert_attn_close(f64(o), want, "block-causal %s" % ((
         B, Lq, Lk, heads, chunk, q_offset, pair, n_split),))
+
+
+# ---------------------------------------------------------------- RoPE --
+
+def _rope_cases(n):
+    cases = []
+    for i in range(n):
+        # token grids up to the RoPE table's side limit on one axis at a
+        # time, a few thousand tokens in all
+        F = int(_RNG.integers(1, 30))
+        H = int(_RNG.integers(1, 40))
+        W = int(_RNG.integers(1, max(2, 4000 // (F * H))))
+        if i % 4 == 3:
+            F, H, W = 1, 1, int(_RNG.integers(900, 1025))  # long width axis
+        B = int(_RNG.integers(1, 3))
+        heads = int(_RNG.integers(1, 17))
+        cases.append(((F, H, W), B, heads, 9500 + 10 * i))
+    return cases
+
+
+@pytest.mark.parametrize(
+    "grid,B,heads,seed", _rope_cases(16),
+    ids=lambda c: "-".join(map(str, c)) if isinstance(c, tuple) else str(c))
+def test_rope_random(grid, B, heads, seed):
+    L = grid[0] * grid[1] * grid[2]
+    q = _bf16((B, L, heads, 128), seed)
+    k = _bf16((B, L, heads, 128), seed + 1)
+    g = wan.grid(*grid)
+    table = wan.rope3d_table(g)
+    qg, kg = cuda(q), cuda(k)
+    wan.rope3d_qk(qg, kg, g, table)
+    torch.cuda.synchronize()
+    assert wan.device_status() == 0
+    for got, x in ((qg, q), (kg, k)):
+        xd = x.double().numpy()
+        want = orope.rope3d(xd, grid)
+        # bf16 output: half an ulp is <= 2^-8 of the value; fp32 arithmetic
+        # and the fp32 table add ~1e-6 of the pair's norm
+        pair = np.repeat(np.sqrt(xd[..., 0::2] ** 2 + xd[..., 1::2] ** 2), 2,
+                         axis=-1)
+        bound = 2.0 ** -8 * np.abs(want) + 1e-6 * pair + 1e-30
+        err = np.abs(got.double().cpu().numpy() - want)
+        assert np.all(err <= bound), (grid, float(np.max(err / bound)))
