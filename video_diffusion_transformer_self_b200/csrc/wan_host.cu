@@ -2,7 +2,9 @@
 // sigma-schedule arithmetic, the RoPE cos/sin table, and the device check.
 #include <math.h>
 
+#include <map>
 #include <mutex>
+#include <utility>
 #include <vector>
 
 #include "wan_internal.cuh"
@@ -25,6 +27,25 @@ int check_device(int* device_out) {
     cached[dev] = (major == 10) ? 1 : 2;
   }
   return cached[dev] == 1 ? WAN_OK : WAN_EUNSUPPORTED;
+}
+
+int resident_grid(const void* kernel, int threads, int dev) {
+  static std::mutex mu;
+  static std::map<std::pair<const void*, int>, int> cache;
+  std::lock_guard<std::mutex> lock(mu);
+  const auto key = std::make_pair(kernel, dev);
+  const auto it = cache.find(key);
+  if (it != cache.end()) return it->second;
+  int sms = 0, per_sm = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+          cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads,
+                                                    0) != cudaSuccess ||
+      sms < 1 || per_sm < 1)
+    return 0;
+  const int grid = sms * (per_sm < 8 ? per_sm : 8);
+  cache[key] = grid;
+  return grid;
 }
 
 namespace {

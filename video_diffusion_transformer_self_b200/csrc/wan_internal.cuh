@@ -19,6 +19,13 @@ namespace wan {
 // else WAN_EUNSUPPORTED / WAN_ECUDA.  Result cached per device.
 int check_device(int* device_out);
 
+// Grid of a grid-stride kernel: the CTAs that can be resident at once on
+// device `dev` (the kernel's occupancy at `threads` threads per CTA, times
+// the SM count), at most 8 per SM, so that no partial last wave runs after
+// the others.  Cached per (kernel, device); returns 0 if the device cannot
+// be queried.
+int resident_grid(const void* kernel, int threads, int dev);
+
 // Tensor map of a [B, L, heads, 128] bf16 tensor with a box of box_rows
 // tokens x 64 channels of one head (dims: channel, head, token, batch),
 // 128-byte swizzle, zero fill past L.
