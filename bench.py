@@ -421,8 +421,14 @@ def causal_rooflines(dev, peak_tflops, reps=5):
         a = off + np.arange(lq, dtype=np.int64)
         return float(np.minimum(L, (a // chunk + 1) * chunk).sum())
 
+    # CTA pairs resident at once (clusters of two CTAs share a GPC, so an SM
+    # left over in a GPC with an odd number of them runs none): the pair
+    # kernel's timings depend on it from box to box
     out = {"workload": "480p-165f", "tokens": L, "heads": H,
-           "chunk_tokens": chunk}
+           "chunk_tokens": chunk,
+           "pair_resident_clusters": wan.attn_pair_resident_clusters(),
+           "sm_count": torch.cuda.get_device_properties(
+               dev).multi_processor_count}
     ql = q[:, L - chunk:].contiguous()
     n_split = wan.block_causal_splits(1, chunk, L, H, chunk, L - chunk)
     ws = torch.empty(max(1, wan.block_causal_workspace_bytes(
