@@ -370,7 +370,8 @@ def hbm_rooflines(dev, g, L, H, n_lat, peak_gbs, n=1 << 30, reps=20):
     cl = torch.randn(n_lat, device=dev, generator=gen)
     ul = torch.randn(n_lat, device=dev, generator=gen)
     tot = 0.0
-    for i in range(reps + 3):
+    cold_reps = 100
+    for i in range(cold_reps + 3):
         flush.fill_(i & 255)
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
@@ -380,8 +381,9 @@ def hbm_rooflines(dev, g, L, H, n_lat, peak_gbs, n=1 << 30, reps=20):
         torch.cuda.synchronize()
         if i >= 3:
             tot += a.elapsed_time(b)
-    ms = tot / reps
+    ms = tot / cold_reps
     out["fm_step_latent_cold"] = {"elements": n_lat, "ms": ms,
+                                  "calls": cold_reps,
                                   "achieved_gbs": 16.0 * n_lat / (ms / 1e3)
                                   / 1e9, "l2": "flushed before each call"}
     return out
@@ -480,7 +482,7 @@ def causal_rooflines(dev, peak_tflops, reps=5):
     return out
 
 
-def attn_points(dev, pk, reps=6):
+def attn_points(dev, pk, reps=10):
     """Self-attention launch alone at the two token counts of the metric:
     480p-81f (B 2 x 12 heads x 32,760 tokens) and 720p-81f (B 1 x 40 heads
     x 75,600 tokens).  Two-tile kernel with Q / K rotated beforehand ("pre"),
@@ -489,10 +491,14 @@ def attn_points(dev, pk, reps=6):
     is the attention alone, the K pass moves half the bytes of the full
     pass); the CTA-pair kernel with Q / K rotated beforehand ("pair_pre") and with Q
     rotated in its tile stage, K by the pass ("pair_fused_q"; the launch
-    timed here is the attention alone).  CUDA events around `reps`
-    back-to-back launches on the launching stream after 2 warm-up launches;
-    Q, K and V are each larger than L2 at 720p (774 MB) and together above
-    it at 480p (3 x 201 MB).  FLOPs 4 * B * heads * L^2 * 128."""
+    timed here is the attention alone).  Each form runs 2 warm-up launches,
+    then `reps` back-to-back launches with a CUDA event on the launching
+    stream between consecutive ones (no idle gap, so each form is timed at
+    the clocks its own steady power draw allows), and reports the median of
+    those launch times (and their mean).  Q, K and V are each larger than
+    L2 at 720p (774 MB) and together above it at 480p (3 x 201 MB).  FLOPs
+    4 * B * heads * L^2 * 128."""
+    import numpy as np
     import torch
 
     from video_diffusion_transformer_self_b200 import wan
@@ -517,35 +523,33 @@ def attn_points(dev, pk, reps=6):
         fl = 4.0 * B * H * L * L * 128
         point = {"tokens": L, "batch": B, "heads": H, "flops": fl}
         wan.rope3d_qk(None, k, g, table)  # k rotated once, for the pair
-        for mode in ("pre", "fused", "fused_q", "pair_pre", "pair_fused_q"):
-            if mode == "pre":
-                def call():
-                    wan.self_attn(q, k, v, o, g)
-            elif mode == "fused":
-                def call():
-                    wan.self_attn(q, k, v, o, g, table=table)
-            elif mode == "fused_q":
-                def call():
-                    wan.self_attn_rope_q(q, k, v, o, g, table)
-            elif mode == "pair_pre":
-                def call():
-                    wan.self_attn_pair(q, k, v, o, g)
-            else:
-                def call():
-                    wan.self_attn_pair(q, k, v, o, g, table_q=table)
+        calls = {
+            "pre": lambda: wan.self_attn(q, k, v, o, g),
+            "fused": lambda: wan.self_attn(q, k, v, o, g, table=table),
+            "fused_q": lambda: wan.self_attn_rope_q(q, k, v, o, g, table),
+            "pair_pre": lambda: wan.self_attn_pair(q, k, v, o, g),
+            "pair_fused_q": lambda: wan.self_attn_pair(q, k, v, o, g,
+                                                       table_q=table),
+        }
+        times = {}
+        for mode, call in calls.items():
             for _ in range(2):
                 call()
-            e0 = torch.cuda.Event(enable_timing=True)
-            e1 = torch.cuda.Event(enable_timing=True)
+            ev = [torch.cuda.Event(enable_timing=True)
+                  for _ in range(reps + 1)]
             torch.cuda.synchronize()
-            e0.record(stream)
-            for _ in range(reps):
+            ev[0].record(stream)
+            for i in range(reps):
                 call()
-            e1.record(stream)
+                ev[i + 1].record(stream)
             torch.cuda.synchronize()
-            ms = e0.elapsed_time(e1) / reps
+            times[mode] = [ev[i].elapsed_time(ev[i + 1]) for i in range(reps)]
+        for mode, t in times.items():
+            ms = float(np.median(t))
             tf = fl / (ms / 1e3) / 1e12
-            point[mode] = {"avg_launch_ms": ms, "tflops": tf,
+            point[mode] = {"median_launch_ms": ms,
+                           "mean_launch_ms": float(np.mean(t)),
+                           "launches": len(t), "tflops": tf,
                            "frac_of_measured_sustained": tf / sustained,
                            "frac_of_measured_burst": tf / burst,
                            "frac_of_datasheet_2250": tf / 2250.0}
