@@ -491,7 +491,7 @@ def attn_points(dev, pk, reps=10):
     is the attention alone, the K pass moves half the bytes of the full
     pass); the CTA-pair kernel with Q / K rotated beforehand ("pair_pre") and with Q
     rotated in its tile stage, K by the pass ("pair_fused_q"; the launch
-    timed here is the attention alone).  Each form runs 2 warm-up launches,
+    timed here is the attention alone).  Each form runs 3 warm-up launches,
     then `reps` back-to-back launches with a CUDA event on the launching
     stream between consecutive ones (no idle gap, so each form is timed at
     the clocks its own steady power draw allows), and reports the median of
@@ -533,7 +533,7 @@ def attn_points(dev, pk, reps=10):
         }
         times = {}
         for mode, call in calls.items():
-            for _ in range(2):
+            for _ in range(3):
                 call()
             ev = [torch.cuda.Event(enable_timing=True)
                   for _ in range(reps + 1)]
